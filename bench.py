@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the EFLA token mixer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ``efla_chunk_fwd`` over the lm340m workload (B=8, H=8,
+L=2048, d=128, bf16 q/k/v, fp32 beta and state, S0 = 0): gate, UT
+transform, state propagation and intra-chunk output all run inside it.
+The headline ``value`` is chunked-forward tokens/s (B*L per step; a token
+carries all H heads) over all ranks, timed on the device with CUDA events.
+The decode metric (batch 64 x 16 heads x d=128, fp32 states) is reported in
+the ``decode`` object of the same line.
+
+Inputs are synthetic and seeded (``workloads``); between timed iterations
+the step rotates over 3 input/output sets (~410 MB, larger than the 126 MB
+L2) so every step reads cold inputs.  Multi-GPU (torchrun, one rank per GPU)
+is weak scaling: every rank runs its own independent (b,h) problems with no
+collective on the data path; time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (test infrastructure) on the
+host cores on a bounded sample of the same workload and prints the same
+line with ``"impl": "reference"``.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+WORKLOAD = "lm340m"
+METRIC = "EFLA chunked-fwd tokens/s (% of tensor/HBM roofline); decode tokens/s"
+ROTATE = 3
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        j = json.load(open(p))
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ algorithmic work
+def chunk_bytes(B, H, L, d, esize, s0: bool, sl: bool = True):
+    """Algorithmic HBM bytes of one efla_chunk_fwd: read q, k, v and beta,
+    write o, read S0 (if given) and write S_L once."""
+    tok = B * H * L
+    state = B * H * d * d * 4
+    return tok * (3 * d * esize + 4 + d * esize) + (state if s0 else 0) + (state if sl else 0)
+
+
+def chunk_flops(B, H, L, d, C=64):
+    """Algorithmic flops of the chunked evaluation per head-token:
+    6 d^2 (W S, K^T D, Q S) + 5 C d (K K^T, Q K^T, W, U, tril(QK^T) D at
+    half density) + C^2/3 (T by forward substitution)."""
+    return B * H * L * (6 * d * d + 5 * C * d + C * C / 3.0)
+
+
+def decode_bytes(B, H, d, esize):
+    return B * H * (2 * 4 * d * d + 4 * d * esize + 4)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Reads SM clock and clock-event reasons through NVML (read-only) every
+    few milliseconds in a background thread; keeps the samples taken while
+    ``active`` is set."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+               0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.active = threading.Event()
+        self.stop_ = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: the line says so
+            self.err = repr(e)
+        self.period = period_s
+        self.th = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_.is_set():
+            if self.active.is_set():
+                try:
+                    self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                    r = get_r(self.h)
+                    for bit, name in self.REASONS.items():
+                        if r & bit and name != "gpu_idle":
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.th.start()
+        return self
+
+    def __exit__(self, *a):
+        self.stop_.set()
+        if self.ok:
+            self.th.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    if world != n_gpus and rank == 0:
+        print(f"note: --gpus {n_gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_rate(x, sample_tokens: int, min_seconds: float, threads: int):
+    """tokens/s of the fp64 oracle on the first ``sample_tokens`` tokens of
+    every (b,h) of ``x`` (a token = one position of one batch row, all heads)."""
+    import oracle
+    B, H = x["q"].shape[:2]
+    sl = lambda t: t[:, :, :sample_tokens].contiguous()
+    q, k, v, beta = (sl(x[n]) for n in ("q", "k", "v", "beta"))
+    oracle.recurrence(q[:1, :1, :8], k[:1, :1, :8], v[:1, :1, :8], beta[:1, :1, :8], threads=1)  # load
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.recurrence(q, k, v, beta, None, threads=threads)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or reps >= 50:
+            break
+    return B * sample_tokens * reps / dt, dt, reps
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle on the host cores."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import oracle
+    w = workloads.WORKLOADS[WORKLOAD]
+    x = workloads.chunk_inputs(w)
+    threads = oracle.default_threads()
+    sample = 64  # one chunk-length of tokens of every (b,h) per step
+    q, k, v, beta = (x[n][:, :, :sample].contiguous() for n in ("q", "k", "v", "beta"))
+    for _ in range(args.warmup):
+        oracle.recurrence(q, k, v, beta, None, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.recurrence(q, k, v, beta, None, threads=threads)
+    dt = time.perf_counter() - t0
+    value = w.B * sample * args.steps / dt
+    desc = (f"fp64 sequential oracle, first {sample} tokens of all {w.B}x{w.H} (b,h) of the {WORKLOAD} "
+            f"workload per step, {threads} threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, workloads.lm340m distribution)",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(w, n):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d={w.d} C=64 {w.dtype} q/k/v, fp32 beta/state, S0=0",
+            "B": w.B, "H": w.H, "L": w.L, "head_dim": w.d, "chunk": 64, "global_batch": w.B * n,
+            "seq_len": w.L, "parallelism": f"dp{n} (independent (b,h) problems per rank, no collective)",
+            "l2": f"inputs/outputs rotate over {ROTATE} sets (> L2) between timed steps"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import delta_rule_linear_03_b200 as efla
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    w = workloads.WORKLOADS[WORKLOAD]
+    B, H, L, d = w.B, w.H, w.L, w.d
+    x = workloads.chunk_inputs(w, seed=42 + w.index + 1000 * rank)
+    sets = []
+    for _ in range(ROTATE):
+        s = {n: x[n].to(dev) for n in ("q", "k", "v", "beta")}
+        s["o"] = torch.empty(B, H, L, d, dtype=x["q"].dtype, device=dev)
+        s["S"] = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+        sets.append(s)
+    need = efla.workspace_size(x["q"].dtype, B, H, L, d, d)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    launches_per_step = 2 if need else 1
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        s = sets[i % ROTATE]
+        efla.chunk_fwd(s["q"], s["k"], s["v"], s["beta"], None, o=s["o"], S_L=s["S"], workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    # capture one CUDA graph per input set so Python launch overhead stays off the clock
+    graphs = []
+    for r in range(ROTATE):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(r)
+        graphs.append(g)
+    for i in range(max(args.warmup, 3)):
+        graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        clk.active.set()
+        e0.record(stream)
+        for i in range(args.steps):
+            graphs[i % ROTATE].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clk.active.clear()
+        barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, world)
+    ms_step = ms_max / args.steps
+    value = world * B * L * args.steps / (ms_max / 1e3)
+    del graphs
+
+    # roofline of the dominant kernel (the whole efla_chunk_fwd when it is one launch)
+    nbytes = chunk_bytes(B, H, L, d, 2, s0=False)
+    flops = chunk_flops(B, H, L, d)
+    achieved_gbs = nbytes / (ms_step / 1e3) / 1e9
+    achieved_tf = flops / (ms_step / 1e3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.lm340m distribution)",
+        "config": workload_config(w, world),
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": achieved_gbs / peaks["hbm"], "traffic": None,
+                     "kernel": "efla_chunk_fwd (all launches of one call)" if launches_per_step > 1
+                     else "efla_chunk_fwd fused kernel",
+                     "algorithmic_bytes": nbytes, "peak_source": peaks["source"]},
+        "roofline_tensor": {"achieved": achieved_tf, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                            "frac": achieved_tf / peaks["bf16"], "algorithmic_flops": flops,
+                            "peak_source": peaks["source"]},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    if rank == 0 and not args.no_decode:
+        line["decode"] = bench_decode(efla, dev, args, peaks)
+    if not args.no_e2e:
+        line["e2e"] = bench_e2e(efla, dev, x, args, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        th = oracle.default_threads()
+        rate, dt, reps = oracle_rate(x, sample_tokens=L, min_seconds=10.0, threads=th)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": th, "kind": "oracle",
+                                "sample": f"full {WORKLOAD} workload x{reps} ({dt:.1f} s), fp64 sequential "
+                                          f"recurrence, OpenMP over (b,h)"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_decode(efla, dev, args, peaks):
+    """Decode: batch 64 x 16 heads x d=128 fp32 states, bf16 q/k/v, one
+    token per step.  Steps rotate over 4 state sets (256 MB > L2) and are
+    replayed from a CUDA graph of 8 steps."""
+    Bd, Hd, d = workloads.DECODE_BATCH, workloads.DECODE_HEADS, 128
+    nsets = 4
+    xin = workloads.decode_inputs(8)
+    ins = [{n: xin[n][i].to(dev) for n in ("q", "k", "v", "beta")} for i in range(8)]
+    states = [workloads.random_state(Bd, Hd, d, seed=s).to(dev) for s in range(nsets)]
+    outs = [torch.empty(Bd, Hd, d, dtype=torch.bfloat16, device=dev) for _ in range(8)]
+
+    def block():
+        for i in range(8):
+            efla.decode_step(ins[i]["q"], ins[i]["k"], ins[i]["v"], ins[i]["beta"], states[i % nsets], o=outs[i])
+
+    for _ in range(3):
+        block()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        block()
+    reps = max(1, args.steps // 8)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_step = e0.elapsed_time(e1) / (8 * reps)
+    nbytes = decode_bytes(Bd, Hd, d, 2)
+    gbs = nbytes / (ms_step / 1e3) / 1e9
+    return {"value": Bd / (ms_step / 1e3), "unit": "tokens/s", "ms_per_step": ms_step, "steps": 8 * reps,
+            "config": f"batch {Bd} x {Hd} heads x d={d}, fp32 states, bf16 q/k/v, {nsets} state sets (> L2)",
+            "gpu_launches": 8 * reps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm"], "traffic": None, "kernel": "decode_kernel",
+                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"]}}
+
+
+def bench_e2e(efla, dev, x, args, world):
+    """The same metric through the public API from pinned host buffers:
+    every step copies q, k, v, beta host->device, runs efla_chunk_fwd and
+    copies o and S_L device->host."""
+    hq, hk, hv, hb = (x[n].pin_memory() for n in ("q", "k", "v", "beta"))
+    B, H, L, d = hq.shape
+    ho = torch.empty(B, H, L, d, dtype=hq.dtype).pin_memory()
+    hS = torch.empty(B, H, d, d, dtype=torch.float32).pin_memory()
+    dq, dk, dv, db = (torch.empty_like(t, device=dev) for t in (hq, hk, hv, hb))
+    do = torch.empty(B, H, L, d, dtype=hq.dtype, device=dev)
+    dS = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+
+    def step():
+        for dst, src in ((dq, hq), (dk, hk), (dv, hv), (db, hb)):
+            dst.copy_(src, non_blocking=True)
+        efla.chunk_fwd(dq, dk, dv, db, None, o=do, S_L=dS)
+        ho.copy_(do, non_blocking=True)
+        hS.copy_(dS, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 30))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record()
+    for _ in range(n):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb))
+    d2h = ho.numel() * ho.element_size() + hS.numel() * hS.element_size()
+    return {"value": world * B * L * n / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

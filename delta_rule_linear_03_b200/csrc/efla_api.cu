@@ -1,0 +1,286 @@
+// efla_api.cu - the C ABI declared in include/efla.h: validation, scratch
+// sizing and kernel dispatch.  Every step of the computation runs in the
+// kernels included below; this file only checks arguments and launches.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/efla.h"
+#include "efla_chunk_simt.cuh"
+#include "efla_chunk_tc.cuh"
+#include "efla_common.cuh"
+#include "efla_decode.cuh"
+#include "efla_gate.cuh"
+
+using namespace efla;
+
+namespace {
+
+constexpr long long kMaxElems = (1LL << 46);  // sanity bound on any tensor's element count
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+size_t esize(efla_dtype_t dt) { return dt == EFLA_F32 ? 4 : 2; }
+
+efla_status_t check_common(efla_dtype_t dtype, efla_mode_t mode) {
+    if (dtype != EFLA_F32 && dtype != EFLA_BF16) return EFLA_ERR_DTYPE;
+    if (mode != EFLA_MODE_EXACT && mode != EFLA_MODE_EULER) return EFLA_ERR_DTYPE;
+    return EFLA_OK;
+}
+
+efla_status_t check_head(int d_k, int d_v) {
+    if (d_k <= 0 || d_v <= 0) return EFLA_ERR_SHAPE;
+    if (d_k != d_v) return EFLA_ERR_UNSUPPORTED;
+    if (d_k != 32 && d_k != 64 && d_k != 128) return EFLA_ERR_UNSUPPORTED;
+    return EFLA_OK;
+}
+
+efla_status_t launched() { return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA; }
+
+// Opt a kernel into more than 48 KB of dynamic shared memory once per
+// device.  Later calls (including ones made while a stream is being
+// captured into a CUDA graph) skip the runtime call.
+template <auto Kernel>
+bool ensure_smem(size_t bytes) {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return false;
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return true;
+}
+
+int num_sms() {
+    static std::atomic<int> cached[64];
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if ((n = cached[dev & 63].load(std::memory_order_relaxed)) > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev & 63].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+template <typename T, int D>
+efla_status_t launch_gate(const void *k, const float *beta, float *alpha, float *lambda, long rows, bool euler,
+                          cudaStream_t st) {
+    constexpr int UNROLL = 4;
+    constexpr int RPW = 32 / (D / (16 / (int)sizeof(T)));
+    const long rows_per_block = 8L * RPW * UNROLL;
+    long blocks = (rows + rows_per_block - 1) / rows_per_block;
+    const long cap = 8L * num_sms();
+    if (blocks > cap) blocks = cap;
+    gate_kernel<T, D, UNROLL><<<(unsigned)blocks, 256, 0, st>>>(static_cast<const T *>(k), beta, alpha, lambda,
+                                                                rows, euler);
+    return launched();
+}
+
+template <typename T, int D>
+efla_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta, float *S, void *o,
+                            long bh, bool euler, cudaStream_t st) {
+    decode_kernel<T, D, D><<<(unsigned)bh, 256, 0, st>>>(static_cast<const T *>(q), static_cast<const T *>(k),
+                                                         static_cast<const T *>(v), beta, S, static_cast<T *>(o),
+                                                         euler);
+    return launched();
+}
+
+template <typename T, int D>
+efla_status_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *beta, const float *S0,
+                                void *o, float *SL, long bh, int L, void *workspace, bool euler, cudaStream_t st) {
+    const int nc = (L + kChunk - 1) / kChunk;
+    const SimtScratch ws = SimtScratch::carve(static_cast<float *>(workspace), bh * nc, D);
+    const size_t prep_smem = sizeof(PrepSmem<D>);
+    const size_t state_smem = sizeof(StateSmem<D>);
+    if (!ensure_smem<chunk_prep_kernel<T, D>>(prep_smem) || !ensure_smem<chunk_state_kernel<T, D>>(state_smem))
+        return EFLA_ERR_CUDA;
+    if ((long long)nc * bh > 0x7fffffffLL) return EFLA_ERR_SHAPE;
+    chunk_prep_kernel<T, D><<<(unsigned)(nc * bh), 256, prep_smem, st>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta, L, nc, ws, euler);
+    if (launched() != EFLA_OK) return EFLA_ERR_CUDA;
+    chunk_state_kernel<T, D><<<(unsigned)((D / StateSmem<D>::DVT) * bh), 256, state_smem, st>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), S0, static_cast<T *>(o), SL, L, nc, ws);
+    return launched();
+}
+
+size_t simt_workspace_bytes(long bh, int L, int d) {
+    const long nc = (L + kChunk - 1) / kChunk;
+    return SimtScratch::floats(bh * nc, d) * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *efla_status_string(efla_status_t s) {
+    switch (s) {
+        case EFLA_OK: return "EFLA_OK";
+        case EFLA_ERR_NULL: return "EFLA_ERR_NULL: a required pointer is NULL";
+        case EFLA_ERR_SHAPE: return "EFLA_ERR_SHAPE: invalid size";
+        case EFLA_ERR_DTYPE: return "EFLA_ERR_DTYPE: unknown dtype or mode";
+        case EFLA_ERR_ALIGN: return "EFLA_ERR_ALIGN: pointer not 16-byte aligned";
+        case EFLA_ERR_UNSUPPORTED: return "EFLA_ERR_UNSUPPORTED: head size must be d_k == d_v in {32,64,128}";
+        case EFLA_ERR_CUDA: return "EFLA_ERR_CUDA: CUDA call or kernel launch failed";
+        case EFLA_ERR_TIMEOUT: return "EFLA_ERR_TIMEOUT: a device-side bounded wait gave up";
+        case EFLA_ERR_WORKSPACE: return "EFLA_ERR_WORKSPACE: workspace missing or too small";
+        case EFLA_ERR_ALIAS: return "EFLA_ERR_ALIAS: an output overlaps an input";
+    }
+    return "EFLA_ERR_UNKNOWN";
+}
+
+int efla_version(void) { return 100; }
+
+efla_status_t efla_last_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return EFLA_ERR_CUDA;
+    unsigned int w = 0;
+    if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return EFLA_ERR_CUDA;
+    if (w) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return EFLA_ERR_CUDA;
+        return EFLA_ERR_TIMEOUT;
+    }
+    return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
+}
+
+efla_status_t efla_gate(const void *k, efla_dtype_t dtype, efla_mode_t mode, const float *beta, float *alpha,
+                        float *lambda, int B, int H, int L, int d_k, efla_stream_t stream) {
+    efla_status_t s = check_common(dtype, mode);
+    if (s != EFLA_OK) return s;
+    if (B < 0 || H < 0 || L < 0 || d_k <= 0) return EFLA_ERR_SHAPE;
+    if ((s = check_head(d_k, d_k)) != EFLA_OK) return s;
+    const long long rows = (long long)B * H * L;
+    if (rows * d_k > kMaxElems) return EFLA_ERR_SHAPE;
+    if (rows == 0) return EFLA_OK;
+    if (!k || !beta || !alpha) return EFLA_ERR_NULL;
+    if (!aligned16(k) || !aligned16(beta) || !aligned16(alpha) || (lambda && !aligned16(lambda)))
+        return EFLA_ERR_ALIGN;
+    const size_t kb = rows * d_k * esize(dtype), rb = rows * sizeof(float);
+    if (overlaps(alpha, rb, k, kb) || overlaps(alpha, rb, beta, rb) || overlaps(lambda, rb, k, kb) ||
+        overlaps(lambda, rb, beta, rb) || overlaps(lambda, rb, alpha, rb))
+        return EFLA_ERR_ALIAS;
+    const bool eu = mode == EFLA_MODE_EULER;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == EFLA_F32) {
+        switch (d_k) {
+            case 32: return launch_gate<float, 32>(k, beta, alpha, lambda, rows, eu, st);
+            case 64: return launch_gate<float, 64>(k, beta, alpha, lambda, rows, eu, st);
+            default: return launch_gate<float, 128>(k, beta, alpha, lambda, rows, eu, st);
+        }
+    }
+    switch (d_k) {
+        case 32: return launch_gate<__nv_bfloat16, 32>(k, beta, alpha, lambda, rows, eu, st);
+        case 64: return launch_gate<__nv_bfloat16, 64>(k, beta, alpha, lambda, rows, eu, st);
+        default: return launch_gate<__nv_bfloat16, 128>(k, beta, alpha, lambda, rows, eu, st);
+    }
+}
+
+size_t efla_chunk_fwd_workspace_size(efla_dtype_t dtype, int B, int H, int L, int d_k, int d_v) {
+    if (check_common(dtype, EFLA_MODE_EXACT) != EFLA_OK || B <= 0 || H <= 0 || L <= 0) return 0;
+    if (check_head(d_k, d_v) != EFLA_OK) return 0;
+    if (tc_path_applies(dtype == EFLA_BF16, d_k, d_v)) return 0;
+    return simt_workspace_bytes((long)B * H, L, d_k);
+}
+
+efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v, efla_dtype_t dtype, efla_mode_t mode,
+                             const float *beta, const float *S0, void *o, float *S_L, int B, int H, int L, int d_k,
+                             int d_v, void *workspace, size_t workspace_bytes, efla_stream_t stream) {
+    efla_status_t s = check_common(dtype, mode);
+    if (s != EFLA_OK) return s;
+    if (B < 0 || H < 0 || L < 0) return EFLA_ERR_SHAPE;
+    if ((s = check_head(d_k, d_v)) != EFLA_OK) return s;
+    const long long bh = (long long)B * H;
+    if (bh * (long long)(L > 0 ? L : 1) * d_k > kMaxElems || bh > 0x7fffffffLL) return EFLA_ERR_SHAPE;
+    if (bh == 0) return EFLA_OK;
+    const size_t sbytes = (size_t)bh * d_k * d_v * sizeof(float);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (L == 0) {  // empty sequence: the state passes through unchanged
+        if (S_L) {
+            if (!aligned16(S_L) || (S0 && !aligned16(S0))) return EFLA_ERR_ALIGN;
+            if (S0 && S0 != S_L && overlaps(S0, sbytes, S_L, sbytes)) return EFLA_ERR_ALIAS;
+            cudaError_t e = S0 ? (S0 == S_L ? cudaSuccess : cudaMemcpyAsync(S_L, S0, sbytes, cudaMemcpyDeviceToDevice, st))
+                               : cudaMemsetAsync(S_L, 0, sbytes, st);
+            return e == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
+        }
+        return EFLA_OK;
+    }
+    if (!q || !k || !v || !beta || !o) return EFLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(o) ||
+        (S0 && !aligned16(S0)) || (S_L && !aligned16(S_L)) || (workspace && !aligned16(workspace)))
+        return EFLA_ERR_ALIGN;
+    const size_t xb = (size_t)bh * L * d_k * esize(dtype), bb = (size_t)bh * L * sizeof(float);
+    if (overlaps(o, xb, q, xb) || overlaps(o, xb, k, xb) || overlaps(o, xb, v, xb) || overlaps(o, xb, beta, bb) ||
+        overlaps(o, xb, S0, sbytes))
+        return EFLA_ERR_ALIAS;
+    if (S_L && (overlaps(S_L, sbytes, q, xb) || overlaps(S_L, sbytes, k, xb) || overlaps(S_L, sbytes, v, xb) ||
+                overlaps(S_L, sbytes, beta, bb) || overlaps(S_L, sbytes, o, xb) ||
+                (S0 && S0 != S_L && overlaps(S_L, sbytes, S0, sbytes))))
+        return EFLA_ERR_ALIAS;
+    const bool eu = mode == EFLA_MODE_EULER;
+    const bool bf = dtype == EFLA_BF16;
+
+    if (tc_path_applies(bf, d_k, d_v))
+        return launch_chunk_tc(q, k, v, beta, S0, o, S_L, bh, L, eu, st);
+
+    const size_t need = simt_workspace_bytes(bh, L, d_k);
+    if (!workspace || workspace_bytes < need) return EFLA_ERR_WORKSPACE;
+    if (overlaps(workspace, need, q, xb) || overlaps(workspace, need, k, xb) || overlaps(workspace, need, v, xb) ||
+        overlaps(workspace, need, o, xb) || overlaps(workspace, need, beta, bb) ||
+        overlaps(workspace, need, S0, sbytes) || overlaps(workspace, need, S_L, sbytes))
+        return EFLA_ERR_ALIAS;
+    if (!bf) {
+        switch (d_k) {
+            case 32: return launch_chunk_simt<float, 32>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
+            case 64: return launch_chunk_simt<float, 64>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
+            default: return launch_chunk_simt<float, 128>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
+        }
+    }
+    switch (d_k) {
+        case 32: return launch_chunk_simt<__nv_bfloat16, 32>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
+        case 64: return launch_chunk_simt<__nv_bfloat16, 64>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
+        default: return launch_chunk_simt<__nv_bfloat16, 128>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
+    }
+}
+
+efla_status_t efla_decode_step(const void *q, const void *k, const void *v, efla_dtype_t dtype, efla_mode_t mode,
+                               const float *beta, float *S, void *o, int B, int H, int d_k, int d_v,
+                               efla_stream_t stream) {
+    efla_status_t s = check_common(dtype, mode);
+    if (s != EFLA_OK) return s;
+    if (B < 0 || H < 0) return EFLA_ERR_SHAPE;
+    if ((s = check_head(d_k, d_v)) != EFLA_OK) return s;
+    const long long bh = (long long)B * H;
+    if (bh * d_k * d_v > kMaxElems || bh > 0x7fffffffLL) return EFLA_ERR_SHAPE;
+    if (bh == 0) return EFLA_OK;
+    if (!q || !k || !v || !beta || !S || !o) return EFLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(S) || !aligned16(o))
+        return EFLA_ERR_ALIGN;
+    const size_t xb = (size_t)bh * d_k * esize(dtype), bb = (size_t)bh * sizeof(float);
+    const size_t sbytes = (size_t)bh * d_k * d_v * sizeof(float);
+    if (overlaps(o, xb, q, xb) || overlaps(o, xb, k, xb) || overlaps(o, xb, v, xb) || overlaps(o, xb, beta, bb) ||
+        overlaps(o, xb, S, sbytes) || overlaps(S, sbytes, q, xb) || overlaps(S, sbytes, k, xb) ||
+        overlaps(S, sbytes, v, xb) || overlaps(S, sbytes, beta, bb))
+        return EFLA_ERR_ALIAS;
+    const bool eu = mode == EFLA_MODE_EULER;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == EFLA_F32) {
+        switch (d_k) {
+            case 32: return launch_decode<float, 32>(q, k, v, beta, S, o, bh, eu, st);
+            case 64: return launch_decode<float, 64>(q, k, v, beta, S, o, bh, eu, st);
+            default: return launch_decode<float, 128>(q, k, v, beta, S, o, bh, eu, st);
+        }
+    }
+    switch (d_k) {
+        case 32: return launch_decode<__nv_bfloat16, 32>(q, k, v, beta, S, o, bh, eu, st);
+        case 64: return launch_decode<__nv_bfloat16, 64>(q, k, v, beta, S, o, bh, eu, st);
+        default: return launch_decode<__nv_bfloat16, 128>(q, k, v, beta, S, o, bh, eu, st);
+    }
+}
+
+}  // extern "C"

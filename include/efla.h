@@ -1,0 +1,159 @@
+/*
+ * efla.h - C ABI of the EFLA (Exact Flow Linear Attention) token mixer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("Exact Flow Linear Attention: Exact Solution from
+ * Continuous-Time Dynamics", papernotes.org summary of arXiv 2512.12602):
+ *
+ *   lambda_t = ||k_t||^2                                   (关键设计 2)
+ *   alpha_t  = (1 - e^{-beta_t lambda_t}) / lambda_t       (关键设计 2)
+ *            = -expm1(-beta_t lc) / lc, lc = max(lambda_t, 1e-12), in fp32
+ *                                                          (损失函数 / 训练策略)
+ *   S_t      = (I - alpha_t k_t k_t^T) S_{t-1} + alpha_t k_t v_t^T
+ *   o_t      = S_t^T q_t                (post-update state; 整体框架 flowchart)
+ *
+ * EFLA_MODE_EULER replaces alpha_t by beta_t, which is the DeltaNet
+ * (explicit Euler) update of section 关键设计 1; everything else is shared.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library allocates nothing; efla_chunk_fwd takes caller-owned scratch.
+ *  - Layouts are dense row-major (C-contiguous):
+ *      q, k      [B][H][L][d_k]       v, o      [B][H][L][d_v]
+ *      beta, alpha, lambda [B][H][L]  (fp32)
+ *      S0, S_L, S          [B][H][d_k][d_v] (fp32)
+ *    For decode L is absent: q,k [B][H][d_k], v,o [B][H][d_v], beta [B][H].
+ *  - q, k, v and o share one storage dtype (efla_dtype_t); beta, alpha,
+ *    lambda and every state are fp32.  Arithmetic is fp32 throughout (the
+ *    bf16 chunk path feeds bf16 operands to tensor-core products that
+ *    accumulate in fp32; the state is kept in fp32).
+ *  - Supported head sizes: d_k == d_v in {32, 64, 128}; anything else
+ *    returns EFLA_ERR_UNSUPPORTED.  B, H >= 0; L >= 0 (L = 0 copies S0 to
+ *    S_L); L need not be a multiple of the internal chunk size.
+ *  - Every pointer must be 16-byte aligned (EFLA_ERR_ALIGN otherwise).
+ *  - Validation is synchronous and happens before anything is enqueued; on
+ *    any error nothing is launched.  Work is enqueued on `stream` and runs
+ *    asynchronously.  Launch failures return EFLA_ERR_CUDA.  Faults that
+ *    happen later on the device surface through efla_last_error() or the
+ *    caller's next synchronising CUDA call.
+ *  - beta may be any real number; NaN and Inf propagate into the outputs
+ *    and are not reported as errors.
+ *  - The calls are thread-safe and keep no host state between calls except
+ *    the sticky device error word read by efla_last_error().
+ */
+#ifndef EFLA_H
+#define EFLA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream.  NULL selects the legacy default stream. */
+typedef struct CUstream_st *efla_stream_t;
+
+typedef enum {
+    EFLA_OK = 0,
+    EFLA_ERR_NULL = 1,        /* a required pointer is NULL                        */
+    EFLA_ERR_SHAPE = 2,       /* a negative size, or an overflowing element count  */
+    EFLA_ERR_DTYPE = 3,       /* unknown efla_dtype_t / efla_mode_t                */
+    EFLA_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned                  */
+    EFLA_ERR_UNSUPPORTED = 5, /* head size outside {32,64,128} or d_k != d_v       */
+    EFLA_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed       */
+    EFLA_ERR_TIMEOUT = 7,     /* a device-side bounded wait gave up (sticky word)  */
+    EFLA_ERR_WORKSPACE = 8,   /* workspace missing or smaller than required        */
+    EFLA_ERR_ALIAS = 9        /* an output overlaps an input it must not overlap   */
+} efla_status_t;
+
+typedef enum { EFLA_F32 = 0, EFLA_BF16 = 1 } efla_dtype_t;
+
+typedef enum {
+    EFLA_MODE_EXACT = 0, /* exact-flow gate alpha_t (EFLA)                 */
+    EFLA_MODE_EULER = 1  /* alpha_t = beta_t (DeltaNet / explicit Euler)   */
+} efla_mode_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *efla_status_string(efla_status_t status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int efla_version(void);
+
+/*
+ * Sticky device error word of the current device.  Synchronises the
+ * current device, returns EFLA_ERR_TIMEOUT if a kernel's bounded wait gave
+ * up since the last call (and clears the word), EFLA_ERR_CUDA if the CUDA
+ * context holds an error, else EFLA_OK.
+ */
+efla_status_t efla_last_error(void);
+
+/*
+ * efla_gate - the exact-flow gate (关键设计 2; numerics per 损失函数 /
+ * 训练策略): for every row t of k,
+ *     lambda[t] = sum_i k[t][i]^2                (fp32 accumulation, unclamped)
+ *     alpha[t]  = -expm1(-beta[t]*lc)/lc,  lc = max(lambda[t], 1e-12)
+ * (alpha[t] = beta[t] in EFLA_MODE_EULER).
+ *   k      [B][H][L][d_k], dtype `dtype`            (input)
+ *   beta   [B][H][L] fp32                            (input)
+ *   alpha  [B][H][L] fp32                            (output)
+ *   lambda [B][H][L] fp32                            (output; may be NULL)
+ * alpha must not overlap k or beta.
+ */
+efla_status_t efla_gate(const void *k, efla_dtype_t dtype, efla_mode_t mode,
+                        const float *beta, float *alpha, float *lambda,
+                        int B, int H, int L, int d_k, efla_stream_t stream);
+
+/*
+ * Bytes of scratch efla_chunk_fwd needs for these sizes (0 if none).  The
+ * value depends only on the arguments.
+ */
+size_t efla_chunk_fwd_workspace_size(efla_dtype_t dtype, int B, int H, int L,
+                                     int d_k, int d_v);
+
+/*
+ * efla_chunk_fwd - prefill over a whole sequence: runs the recurrence above
+ * for t = 0..L-1 from S0 and writes every o_t and the final state.  It
+ * evaluates the recurrence chunk by chunk in the UT form of the chunked
+ * scheme the pages cite (整体框架: "WY / UT" chunk-parallel products):
+ *     A = strictly-lower(diag(alpha) K K^T),  T = (I + A)^{-1},
+ *     W = T diag(alpha) K,  U = T diag(alpha) V,
+ *     D = U - W S,  O = Q S + lower-incl-diag(Q K^T) D,  S <- S + K^T D,
+ * which equals the token-by-token recurrence up to rounding.
+ *   q, k  [B][H][L][d_k]   v [B][H][L][d_v]   dtype `dtype`   (inputs)
+ *   beta  [B][H][L] fp32                                        (input)
+ *   S0    [B][H][d_k][d_v] fp32, or NULL for the zero state     (input)
+ *   o     [B][H][L][d_v] dtype `dtype`                          (output)
+ *   S_L   [B][H][d_k][d_v] fp32, or NULL if not wanted          (output)
+ *   workspace / workspace_bytes: caller-owned device scratch of at least
+ *     efla_chunk_fwd_workspace_size(...) bytes (may be NULL when that is 0);
+ *     its contents on entry are ignored and on exit undefined.
+ * S_L may be the same pointer as S0 (in-place state update).  o must not
+ * overlap any input; S_L must not overlap q, k, v, beta or o.
+ */
+efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v,
+                             efla_dtype_t dtype, efla_mode_t mode,
+                             const float *beta, const float *S0, void *o,
+                             float *S_L, int B, int H, int L, int d_k, int d_v,
+                             void *workspace, size_t workspace_bytes,
+                             efla_stream_t stream);
+
+/*
+ * efla_decode_step - one token of the recurrence for B*H independent
+ * states, updated in place:
+ *     S <- (I - alpha k k^T) S + alpha k v^T,   o = S^T q  (updated S)
+ *   q, k [B][H][d_k]   v [B][H][d_v]   dtype `dtype`   (inputs)
+ *   beta [B][H] fp32                                    (input)
+ *   S    [B][H][d_k][d_v] fp32                          (input/output)
+ *   o    [B][H][d_v] dtype `dtype`                      (output)
+ * o must not overlap S or any input.
+ */
+efla_status_t efla_decode_step(const void *q, const void *k, const void *v,
+                               efla_dtype_t dtype, efla_mode_t mode,
+                               const float *beta, float *S, void *o, int B,
+                               int H, int d_k, int d_v, efla_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EFLA_H */

@@ -1,0 +1,97 @@
+"""The C-ABI library loads and exports every call include/efla.h declares,
+and its synchronous argument validation rejects bad calls before touching
+a GPU (no compute calls here; these run on a CPU-only machine)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "efla.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(efla_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import delta_rule_linear_03_b200 as efla
+    return efla._lib, efla
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("efla_gate", "efla_chunk_fwd", "efla_decode_step"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so, efla = lib
+    for name in declared_functions():
+        assert hasattr(so, name), f"libefla.so does not export {name}"
+
+
+def test_status_strings_and_version(lib):
+    so, efla = lib
+    assert efla.version() >= 100
+    for code, name in efla.STATUS.items():
+        assert so.efla_status_string(code).decode().startswith(name)
+
+
+A = ctypes.c_void_p(0x10000)  # aligned fake device addresses: never dereferenced
+A2 = ctypes.c_void_p(0x20000)
+A3 = ctypes.c_void_p(0x30000)
+A4 = ctypes.c_void_p(0x40000)
+A5 = ctypes.c_void_p(0x50000)
+A6 = ctypes.c_void_p(0x60000)
+
+
+def test_validation_rejects_before_launch(lib):
+    so, efla = lib
+    F32, BF16 = 0, 1
+    # bad dtype / mode
+    assert so.efla_chunk_fwd(A, A2, A3, 7, 0, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 3
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 9, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 3
+    # unsupported head sizes
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 48, 48, None, 0, None) == 5
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 128, 64, None, 0, None) == 5
+    assert so.efla_decode_step(A, A2, A3, F32, 0, A4, A5, A6, 1, 1, 256, 256, None) == 5
+    # negative sizes
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, None, -1, 1, 64, 128, 128, None, 0, None) == 2
+    assert so.efla_gate(A, F32, 0, A2, A3, None, 1, 1, -5, 128, None) == 2
+    # NULL required pointers
+    assert so.efla_chunk_fwd(None, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 1
+    assert so.efla_decode_step(A, A2, A3, BF16, 0, A4, None, A6, 1, 1, 128, 128, None) == 1
+    assert so.efla_gate(None, F32, 0, A2, A3, None, 1, 1, 5, 128, None) == 1
+    # misaligned pointers
+    bad = ctypes.c_void_p(0x10004)
+    assert so.efla_chunk_fwd(bad, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 4
+    assert so.efla_decode_step(A, A2, A3, F32, 0, A4, bad, A6, 1, 1, 128, 128, None) == 4
+    # aliasing: o on top of q
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A, None, 1, 1, 64, 128, 128, None, 0, None) == 9
+    # workspace required for the fp32 path and absent
+    need = so.efla_chunk_fwd_workspace_size(F32, 1, 1, 64, 128, 128)
+    assert need > 0
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 8
+    # empty problems are accepted without any launch
+    assert so.efla_chunk_fwd(None, None, None, F32, 0, None, None, None, None, 0, 4, 64, 128, 128, None, 0,
+                             None) == 0
+    assert so.efla_decode_step(None, None, None, F32, 0, None, None, None, 3, 0, 64, 64, None) == 0
+    assert so.efla_gate(None, F32, 0, None, None, None, 2, 2, 0, 32, None) == 0
+    # L = 0 without S_L: nothing to do
+    assert so.efla_chunk_fwd(None, None, None, BF16, 0, None, None, None, None, 2, 2, 0, 64, 64, None, 0,
+                             None) == 0
+
+
+def test_workspace_size_is_pure_and_scales(lib):
+    so, _ = lib
+    a = so.efla_chunk_fwd_workspace_size(0, 2, 16, 8192, 128, 128)
+    b = so.efla_chunk_fwd_workspace_size(0, 2, 16, 8192, 128, 128)
+    assert a == b and a > 0
+    assert so.efla_chunk_fwd_workspace_size(0, 4, 16, 8192, 128, 128) == 2 * a
+    assert so.efla_chunk_fwd_workspace_size(0, 2, 16, 8192, 48, 48) == 0
+    assert so.efla_chunk_fwd_workspace_size(0, 0, 16, 8192, 128, 128) == 0

@@ -1,0 +1,154 @@
+"""efla_chunk_fwd on the GPU against the sequential fp64 oracle.
+
+Sizes here finish in seconds in the oracle yet span several 64-token
+chunks and a ragged tail; the full workload sizes are in
+test_gpu_fullsize.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import assert_close, np64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def efla():
+    import delta_rule_linear_03_b200 as m
+    return m
+
+
+def run(efla, x, mode="exact", S0=None):
+    o, SL = efla.chunk_fwd(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), x["beta"].cuda(),
+                           None if S0 is None else S0.cuda(), mode=mode)
+    torch.cuda.synchronize()
+    return o, SL
+
+
+def ref(x, mode="exact", S0=None):
+    return oracle.recurrence(x["q"], x["k"], x["v"], x["beta"], S0, euler=(mode == "euler"))
+
+
+@pytest.mark.parametrize("mode", ["exact", "euler"])
+def test_tiny_full(efla, mode):
+    x = workloads.chunk_inputs("tiny_d32")
+    o, SL = run(efla, x, mode)
+    ro, rS = ref(x, mode)
+    assert_close(o, ro, "f32", "o")
+    assert_close(SL, rS, "f32", "S_L")
+
+
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 200, 333])
+def test_lm_ragged_lengths(efla, L):
+    x = workloads.chunk_inputs("lm340m", B=2, H=3, L=L)
+    o, SL = run(efla, x)
+    ro, rS = ref(x)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(SL, rS, "bf16", "S_L")
+
+
+def test_lm_with_initial_state(efla):
+    x = workloads.chunk_inputs("lm1p3b", B=2, H=4, L=517)
+    o, SL = run(efla, x, S0=x["S0"])
+    ro, rS = ref(x, S0=x["S0"])
+    assert_close(o, ro, "bf16", "o")
+    assert_close(SL, rS, "bf16", "S_L")
+
+
+@pytest.mark.parametrize("knorm", workloads.STIFF_KNORMS)
+def test_stiffness_reduced(efla, knorm):
+    x = workloads.chunk_inputs("stiffness", B=1, H=4, L=700, knorm=knorm)
+    o, SL = run(efla, x)
+    ro, rS = ref(x)
+    assert_close(o, ro, "f32", "o")
+    assert_close(SL, rS, "f32", "S_L")
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_head_sizes(efla, d, dtype):
+    g = torch.Generator().manual_seed(d)
+    B, H, L = 2, 2, 150
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    x = dict(q=torch.randn(B, H, L, d, generator=g).to(tdt),
+             k=(torch.randn(B, H, L, d, generator=g) / d ** 0.5).to(tdt),
+             v=torch.randn(B, H, L, d, generator=g).to(tdt),
+             beta=torch.rand(B, H, L, generator=g))
+    S0 = torch.randn(B, H, d, d, generator=g) * 0.1
+    o, SL = run(efla, x, S0=S0)
+    ro, rS = ref(x, S0=S0)
+    assert_close(o, ro, dtype, "o")
+    assert_close(SL, rS, dtype, "S_L")
+
+
+def test_split_sequence_chaining(efla):
+    """chunk_fwd over L equals chunk_fwd over L1 then over L - L1 from S_L1,
+    for a split that is not a multiple of the chunk size (checkpoint/resume)."""
+    x = workloads.chunk_inputs("tiny_d32", L=256)
+    L1 = 100
+    a = {k: v[:, :, :L1] for k, v in x.items() if v is not None}
+    b = {k: v[:, :, L1:] for k, v in x.items() if v is not None}
+    o1, S1 = run(efla, a)
+    o2, S2 = efla.chunk_fwd(b["q"].cuda(), b["k"].cuda(), b["v"].cuda(), b["beta"].cuda(), S1)
+    ro, rS = ref(x)
+    assert_close(torch.cat([o1, o2], dim=2), ro, "f32", "o")
+    assert_close(S2, rS, "f32", "S_L")
+
+
+def test_in_place_state(efla):
+    x = workloads.chunk_inputs("tiny_d32", L=130)
+    S = torch.randn(1, 2, 32, 32) * 0.3
+    Sg = S.cuda()
+    o, SL = efla.chunk_fwd(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), x["beta"].cuda(), Sg, S_L=Sg)
+    torch.cuda.synchronize()
+    assert SL.data_ptr() == Sg.data_ptr()
+    ro, rS = ref(x, S0=S)
+    assert_close(o, ro, "f32", "o")
+    assert_close(Sg, rS, "f32", "S_L")
+
+
+def test_empty_sequence_passes_state_through(efla):
+    S0 = torch.randn(2, 3, 64, 64, device="cuda")
+    z = torch.empty(2, 3, 0, 64, device="cuda")
+    o, SL = efla.chunk_fwd(z, z, z, torch.empty(2, 3, 0, device="cuda"), S0)
+    torch.cuda.synchronize()
+    assert o.shape == (2, 3, 0, 64)
+    assert torch.equal(SL, S0)
+    o, SL = efla.chunk_fwd(z, z, z, torch.empty(2, 3, 0, device="cuda"), None)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(SL) == 0
+
+
+def test_zero_beta_is_identity(efla):
+    x = workloads.chunk_inputs("tiny_d32", L=90)
+    x["beta"] = torch.zeros_like(x["beta"])
+    S0 = torch.randn(1, 2, 32, 32)
+    o, SL = run(efla, x, S0=S0)
+    np.testing.assert_allclose(np64(SL), np64(S0), atol=0)
+    ro, _ = ref(x, S0=S0)
+    assert_close(o, ro, "f32", "o")
+
+
+def test_workspace_too_small_is_rejected(efla):
+    x = workloads.chunk_inputs("tiny_d32", L=128)
+    need = efla.workspace_size(torch.float32, 1, 2, 128, 32, 32)
+    ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    import ctypes
+    o = torch.empty(1, 2, 128, 32, device="cuda")
+    st = efla._lib.efla_chunk_fwd(*(ctypes.c_void_p(t.data_ptr()) for t in (x["q"].cuda(), x["k"].cuda(),
+                                                                            x["v"].cuda())),
+                                  0, 0, ctypes.c_void_p(x["beta"].cuda().data_ptr()), None,
+                                  ctypes.c_void_p(o.data_ptr()), None, 1, 2, 128, 32, 32,
+                                  ctypes.c_void_p(ws.data_ptr()), need - 16, None)
+    assert st == 8
+    assert efla.last_error() == 0
+
+
+def test_repeatable(efla):
+    """Two identical calls give bit-identical results (no races)."""
+    x = workloads.chunk_inputs("lm340m", B=2, H=2, L=300)
+    o1, S1 = run(efla, x)
+    o2, S2 = run(efla, x)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
