@@ -56,12 +56,12 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ algorithmic work
-def chunk_bytes(B, H, L, d, esize, s0: bool, sl: bool = True):
+def chunk_bytes(B, H, L, d, esize, esize_o, s0: bool, sl: bool = True):
     """Algorithmic HBM bytes of one efla_chunk_fwd: read q, k, v and beta,
     write o, read S0 (if given) and write S_L once."""
     tok = B * H * L
     state = B * H * d * d * 4
-    return tok * (3 * d * esize + 4 + d * esize) + (state if s0 else 0) + (state if sl else 0)
+    return tok * (3 * d * esize + 4 + d * esize_o) + (state if s0 else 0) + (state if sl else 0)
 
 
 def chunk_flops(B, H, L, d, C=64):
@@ -71,8 +71,9 @@ def chunk_flops(B, H, L, d, C=64):
     return B * H * L * (6 * d * d + 5 * C * d + C * C / 3.0)
 
 
-def decode_bytes(B, H, d, esize):
-    return B * H * (2 * 4 * d * d + 4 * d * esize + 4)
+def decode_bytes(B, H, d, esize, esize_o):
+    """Read and write the fp32 state once, read q, k, v and beta, write o."""
+    return B * H * (2 * 4 * d * d + 3 * d * esize + 4 + d * esize_o)
 
 
 # ------------------------------------------------------------------ clocks
@@ -227,7 +228,7 @@ def run_reference(args):
 
 
 def workload_config(w, n):
-    return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d={w.d} C=64 {w.dtype} q/k/v, fp32 beta/state, S0=0",
+    return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d={w.d} C=64 {w.dtype} q/k/v, fp32 beta/state/o, S0=0",
             "B": w.B, "H": w.H, "L": w.L, "head_dim": w.d, "chunk": 64, "global_batch": w.B * n,
             "seq_len": w.L, "parallelism": f"dp{n} (independent (b,h) problems per rank, no collective)",
             "l2": f"inputs/outputs rotate over {ROTATE} sets (> L2) between timed steps"}
@@ -246,7 +247,7 @@ def run_ours(args):
     sets = []
     for _ in range(ROTATE):
         s = {n: x[n].to(dev) for n in ("q", "k", "v", "beta")}
-        s["o"] = torch.empty(B, H, L, d, dtype=x["q"].dtype, device=dev)
+        s["o"] = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
         s["S"] = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
         sets.append(s)
     need = efla.workspace_size(x["q"].dtype, B, H, L, d, d)
@@ -291,7 +292,7 @@ def run_ours(args):
     del graphs
 
     # roofline of the dominant kernel (the whole efla_chunk_fwd when it is one launch)
-    nbytes = chunk_bytes(B, H, L, d, 2, s0=False)
+    nbytes = chunk_bytes(B, H, L, d, 2, 4, s0=False)
     flops = chunk_flops(B, H, L, d)
     achieved_gbs = nbytes / (ms_step / 1e3) / 1e9
     achieved_tf = flops / (ms_step / 1e3) / 1e12
@@ -344,7 +345,7 @@ def bench_decode(efla, dev, args, peaks):
     xin = workloads.decode_inputs(8)
     ins = [{n: xin[n][i].to(dev) for n in ("q", "k", "v", "beta")} for i in range(8)]
     states = [workloads.random_state(Bd, Hd, d, seed=s).to(dev) for s in range(nsets)]
-    outs = [torch.empty(Bd, Hd, d, dtype=torch.bfloat16, device=dev) for _ in range(8)]
+    outs = [torch.empty(Bd, Hd, d, dtype=torch.float32, device=dev) for _ in range(8)]
 
     def block():
         for i in range(8):
@@ -367,10 +368,10 @@ def bench_decode(efla, dev, args, peaks):
     e1.record()
     torch.cuda.synchronize()
     ms_step = e0.elapsed_time(e1) / (8 * reps)
-    nbytes = decode_bytes(Bd, Hd, d, 2)
+    nbytes = decode_bytes(Bd, Hd, d, 2, 4)
     gbs = nbytes / (ms_step / 1e3) / 1e9
     return {"value": Bd / (ms_step / 1e3), "unit": "tokens/s", "ms_per_step": ms_step, "steps": 8 * reps,
-            "config": f"batch {Bd} x {Hd} heads x d={d}, fp32 states, bf16 q/k/v, {nsets} state sets (> L2)",
+            "config": f"batch {Bd} x {Hd} heads x d={d}, fp32 states, bf16 q/k/v, fp32 o, {nsets} state sets (> L2)",
             "gpu_launches": 8 * reps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm"], "traffic": None, "kernel": "decode_kernel",
@@ -383,10 +384,10 @@ def bench_e2e(efla, dev, x, args, world):
     copies o and S_L device->host."""
     hq, hk, hv, hb = (x[n].pin_memory() for n in ("q", "k", "v", "beta"))
     B, H, L, d = hq.shape
-    ho = torch.empty(B, H, L, d, dtype=hq.dtype).pin_memory()
+    ho = torch.empty(B, H, L, d, dtype=torch.float32).pin_memory()
     hS = torch.empty(B, H, d, d, dtype=torch.float32).pin_memory()
     dq, dk, dv, db = (torch.empty_like(t, device=dev) for t in (hq, hk, hv, hb))
-    do = torch.empty(B, H, L, d, dtype=hq.dtype, device=dev)
+    do = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
     dS = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
 
     def step():

@@ -54,9 +54,9 @@ _lib.efla_gate.argtypes = [_p, _i, _i, _p, _p, _p, _i, _i, _i, _i, _p]
 _lib.efla_chunk_fwd_workspace_size.restype = _sz
 _lib.efla_chunk_fwd_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
 _lib.efla_chunk_fwd.restype = _i
-_lib.efla_chunk_fwd.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _sz, _p]
+_lib.efla_chunk_fwd.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _p, _sz, _p]
 _lib.efla_decode_step.restype = _i
-_lib.efla_decode_step.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _i, _i, _i, _p]
+_lib.efla_decode_step.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 
 
 class EflaError(RuntimeError):
@@ -133,10 +133,11 @@ def workspace_size(dtype: torch.dtype, B: int, H: int, L: int, d_k: int, d_v: in
 
 
 def chunk_fwd(q, k, v, beta, S0=None, mode: str = "exact", o=None, S_L=None, want_state: bool = True,
-              workspace=None):
+              workspace=None, out_dtype=torch.float32):
     """Prefill: q,k [B,H,L,d_k], v [B,H,L,d_v] (one dtype, fp32 or bf16), beta [B,H,L]
-    fp32, S0 [B,H,d_k,d_v] fp32 or None.  Returns (o [B,H,L,d_v] in q's dtype,
-    S_L [B,H,d_k,d_v] fp32 or None).  ``S_L=S0`` updates the state in place."""
+    fp32, S0 [B,H,d_k,d_v] fp32 or None.  Returns (o [B,H,L,d_v] in ``out_dtype``
+    (or ``o.dtype`` when ``o`` is given), S_L [B,H,d_k,d_v] fp32 or None).
+    ``S_L=S0`` updates the state in place."""
     dev = _dev(q, k, v, beta, S0)
     B, H, L, dk = k.shape
     dv = v.shape[-1]
@@ -146,7 +147,9 @@ def chunk_fwd(q, k, v, beta, S0=None, mode: str = "exact", o=None, S_L=None, wan
         raise ValueError("beta must be float32 [B,H,L]")
     if S0 is not None and (S0.dtype != torch.float32 or tuple(S0.shape) != (B, H, dk, dv)):
         raise ValueError("S0 must be float32 [B,H,d_k,d_v]")
-    o = torch.empty((B, H, L, dv), dtype=q.dtype, device=dev) if o is None else o
+    o = torch.empty((B, H, L, dv), dtype=out_dtype, device=dev) if o is None else o
+    if tuple(o.shape) != (B, H, L, dv):
+        raise ValueError("o must be [B,H,L,d_v]")
     if want_state and S_L is None:
         S_L = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     _dev(o, S_L)
@@ -156,15 +159,16 @@ def chunk_fwd(q, k, v, beta, S0=None, mode: str = "exact", o=None, S_L=None, wan
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
         _check(_lib.efla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _dt(q), MODES[mode], _ptr(beta), _ptr(S0),
-                                   _ptr(o), _ptr(S_L), B, H, L, dk, dv,
+                                   _ptr(o), _dt(o), _ptr(S_L), B, H, L, dk, dv,
                                    _ptr(workspace) if need else None, wbytes if need else 0,
                                    _stream(dev)), "efla_chunk_fwd")
     return o, S_L
 
 
-def decode_step(q, k, v, beta, S, mode: str = "exact", o=None):
+def decode_step(q, k, v, beta, S, mode: str = "exact", o=None, out_dtype=torch.float32):
     """One token for B*H states: q,k [B,H,d_k], v [B,H,d_v], beta [B,H] fp32,
-    S [B,H,d_k,d_v] fp32 updated in place.  Returns o [B,H,d_v] in q's dtype."""
+    S [B,H,d_k,d_v] fp32 updated in place.  Returns o [B,H,d_v] in ``out_dtype``
+    (or ``o.dtype`` when ``o`` is given)."""
     dev = _dev(q, k, v, beta, S)
     B, H, dk = k.shape
     dv = v.shape[-1]
@@ -174,9 +178,11 @@ def decode_step(q, k, v, beta, S, mode: str = "exact", o=None):
         raise ValueError("beta must be float32 [B,H]")
     if S.dtype != torch.float32 or tuple(S.shape) != (B, H, dk, dv):
         raise ValueError("S must be float32 [B,H,d_k,d_v]")
-    o = torch.empty((B, H, dv), dtype=q.dtype, device=dev) if o is None else o
+    o = torch.empty((B, H, dv), dtype=out_dtype, device=dev) if o is None else o
+    if tuple(o.shape) != (B, H, dv):
+        raise ValueError("o must be [B,H,d_v]")
     _dev(o)
     with torch.cuda.device(dev):
         _check(_lib.efla_decode_step(_ptr(q), _ptr(k), _ptr(v), _dt(q), MODES[mode], _ptr(beta), _ptr(S),
-                                     _ptr(o), B, H, dk, dv, _stream(dev)), "efla_decode_step")
+                                     _ptr(o), _dt(o), B, H, dk, dv, _stream(dev)), "efla_decode_step")
     return o

@@ -83,30 +83,30 @@ efla_status_t launch_gate(const void *k, const float *beta, float *alpha, float 
     return launched();
 }
 
-template <typename T, int D>
+template <typename T, typename To, int D>
 efla_status_t launch_decode(const void *q, const void *k, const void *v, const float *beta, float *S, void *o,
                             long bh, bool euler, cudaStream_t st) {
-    decode_kernel<T, D, D><<<(unsigned)bh, 256, 0, st>>>(static_cast<const T *>(q), static_cast<const T *>(k),
-                                                         static_cast<const T *>(v), beta, S, static_cast<T *>(o),
-                                                         euler);
+    decode_kernel<T, To, D, D><<<(unsigned)bh, 256, 0, st>>>(static_cast<const T *>(q), static_cast<const T *>(k),
+                                                             static_cast<const T *>(v), beta, S,
+                                                             static_cast<To *>(o), euler);
     return launched();
 }
 
-template <typename T, int D>
+template <typename T, typename To, int D>
 efla_status_t launch_chunk_simt(const void *q, const void *k, const void *v, const float *beta, const float *S0,
                                 void *o, float *SL, long bh, int L, void *workspace, bool euler, cudaStream_t st) {
     const int nc = (L + kChunk - 1) / kChunk;
     const SimtScratch ws = SimtScratch::carve(static_cast<float *>(workspace), bh * nc, D);
     const size_t prep_smem = sizeof(PrepSmem<D>);
     const size_t state_smem = sizeof(StateSmem<D>);
-    if (!ensure_smem<chunk_prep_kernel<T, D>>(prep_smem) || !ensure_smem<chunk_state_kernel<T, D>>(state_smem))
+    if (!ensure_smem<chunk_prep_kernel<T, D>>(prep_smem) || !ensure_smem<chunk_state_kernel<T, To, D>>(state_smem))
         return EFLA_ERR_CUDA;
     if ((long long)nc * bh > 0x7fffffffLL) return EFLA_ERR_SHAPE;
     chunk_prep_kernel<T, D><<<(unsigned)(nc * bh), 256, prep_smem, st>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta, L, nc, ws, euler);
     if (launched() != EFLA_OK) return EFLA_ERR_CUDA;
-    chunk_state_kernel<T, D><<<(unsigned)((D / StateSmem<D>::DVT) * bh), 256, state_smem, st>>>(
-        static_cast<const T *>(q), static_cast<const T *>(k), S0, static_cast<T *>(o), SL, L, nc, ws);
+    chunk_state_kernel<T, To, D><<<(unsigned)((D / StateSmem<D>::DVT) * bh), 256, state_smem, st>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), S0, static_cast<To *>(o), SL, L, nc, ws);
     return launched();
 }
 
@@ -114,6 +114,30 @@ size_t simt_workspace_bytes(long bh, int L, int d) {
     const long nc = (L + kChunk - 1) / kChunk;
     return SimtScratch::floats(bh * nc, d) * sizeof(float);
 }
+
+// Instantiate F<Tin, Tout, D>(args...) for the runtime (dtype, o_dtype, d).
+#define EFLA_DISPATCH(F, dtype, odtype, d, ...)                                                   \
+    do {                                                                                          \
+        const bool bf_in_ = (dtype) == EFLA_BF16, bf_out_ = (odtype) == EFLA_BF16;                \
+        if (!bf_in_ && !bf_out_) {                                                                \
+            if ((d) == 32) return F<float, float, 32>(__VA_ARGS__);                               \
+            if ((d) == 64) return F<float, float, 64>(__VA_ARGS__);                               \
+            return F<float, float, 128>(__VA_ARGS__);                                             \
+        }                                                                                         \
+        if (!bf_in_ && bf_out_) {                                                                 \
+            if ((d) == 32) return F<float, __nv_bfloat16, 32>(__VA_ARGS__);                       \
+            if ((d) == 64) return F<float, __nv_bfloat16, 64>(__VA_ARGS__);                       \
+            return F<float, __nv_bfloat16, 128>(__VA_ARGS__);                                     \
+        }                                                                                         \
+        if (bf_in_ && !bf_out_) {                                                                 \
+            if ((d) == 32) return F<__nv_bfloat16, float, 32>(__VA_ARGS__);                       \
+            if ((d) == 64) return F<__nv_bfloat16, float, 64>(__VA_ARGS__);                       \
+            return F<__nv_bfloat16, float, 128>(__VA_ARGS__);                                     \
+        }                                                                                         \
+        if ((d) == 32) return F<__nv_bfloat16, __nv_bfloat16, 32>(__VA_ARGS__);                   \
+        if ((d) == 64) return F<__nv_bfloat16, __nv_bfloat16, 64>(__VA_ARGS__);                   \
+        return F<__nv_bfloat16, __nv_bfloat16, 128>(__VA_ARGS__);                                 \
+    } while (0)
 
 }  // namespace
 
@@ -189,10 +213,12 @@ size_t efla_chunk_fwd_workspace_size(efla_dtype_t dtype, int B, int H, int L, in
 }
 
 efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v, efla_dtype_t dtype, efla_mode_t mode,
-                             const float *beta, const float *S0, void *o, float *S_L, int B, int H, int L, int d_k,
-                             int d_v, void *workspace, size_t workspace_bytes, efla_stream_t stream) {
+                             const float *beta, const float *S0, void *o, efla_dtype_t o_dtype, float *S_L, int B,
+                             int H, int L, int d_k, int d_v, void *workspace, size_t workspace_bytes,
+                             efla_stream_t stream) {
     efla_status_t s = check_common(dtype, mode);
     if (s != EFLA_OK) return s;
+    if ((s = check_common(o_dtype, mode)) != EFLA_OK) return s;
     if (B < 0 || H < 0 || L < 0) return EFLA_ERR_SHAPE;
     if ((s = check_head(d_k, d_v)) != EFLA_OK) return s;
     const long long bh = (long long)B * H;
@@ -215,44 +241,35 @@ efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v, efla_d
         (S0 && !aligned16(S0)) || (S_L && !aligned16(S_L)) || (workspace && !aligned16(workspace)))
         return EFLA_ERR_ALIGN;
     const size_t xb = (size_t)bh * L * d_k * esize(dtype), bb = (size_t)bh * L * sizeof(float);
-    if (overlaps(o, xb, q, xb) || overlaps(o, xb, k, xb) || overlaps(o, xb, v, xb) || overlaps(o, xb, beta, bb) ||
-        overlaps(o, xb, S0, sbytes))
+    const size_t ob = (size_t)bh * L * d_v * esize(o_dtype);
+    if (overlaps(o, ob, q, xb) || overlaps(o, ob, k, xb) || overlaps(o, ob, v, xb) || overlaps(o, ob, beta, bb) ||
+        overlaps(o, ob, S0, sbytes))
         return EFLA_ERR_ALIAS;
     if (S_L && (overlaps(S_L, sbytes, q, xb) || overlaps(S_L, sbytes, k, xb) || overlaps(S_L, sbytes, v, xb) ||
-                overlaps(S_L, sbytes, beta, bb) || overlaps(S_L, sbytes, o, xb) ||
+                overlaps(S_L, sbytes, beta, bb) || overlaps(S_L, sbytes, o, ob) ||
                 (S0 && S0 != S_L && overlaps(S_L, sbytes, S0, sbytes))))
         return EFLA_ERR_ALIAS;
     const bool eu = mode == EFLA_MODE_EULER;
     const bool bf = dtype == EFLA_BF16;
 
     if (tc_path_applies(bf, d_k, d_v))
-        return launch_chunk_tc(q, k, v, beta, S0, o, S_L, bh, L, eu, st);
+        return launch_chunk_tc(q, k, v, beta, S0, o, o_dtype == EFLA_BF16, S_L, bh, L, eu, st);
 
     const size_t need = simt_workspace_bytes(bh, L, d_k);
     if (!workspace || workspace_bytes < need) return EFLA_ERR_WORKSPACE;
     if (overlaps(workspace, need, q, xb) || overlaps(workspace, need, k, xb) || overlaps(workspace, need, v, xb) ||
-        overlaps(workspace, need, o, xb) || overlaps(workspace, need, beta, bb) ||
+        overlaps(workspace, need, o, ob) || overlaps(workspace, need, beta, bb) ||
         overlaps(workspace, need, S0, sbytes) || overlaps(workspace, need, S_L, sbytes))
         return EFLA_ERR_ALIAS;
-    if (!bf) {
-        switch (d_k) {
-            case 32: return launch_chunk_simt<float, 32>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
-            case 64: return launch_chunk_simt<float, 64>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
-            default: return launch_chunk_simt<float, 128>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
-        }
-    }
-    switch (d_k) {
-        case 32: return launch_chunk_simt<__nv_bfloat16, 32>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
-        case 64: return launch_chunk_simt<__nv_bfloat16, 64>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
-        default: return launch_chunk_simt<__nv_bfloat16, 128>(q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
-    }
+    EFLA_DISPATCH(launch_chunk_simt, dtype, o_dtype, d_k, q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
 }
 
 efla_status_t efla_decode_step(const void *q, const void *k, const void *v, efla_dtype_t dtype, efla_mode_t mode,
-                               const float *beta, float *S, void *o, int B, int H, int d_k, int d_v,
-                               efla_stream_t stream) {
+                               const float *beta, float *S, void *o, efla_dtype_t o_dtype, int B, int H, int d_k,
+                               int d_v, efla_stream_t stream) {
     efla_status_t s = check_common(dtype, mode);
     if (s != EFLA_OK) return s;
+    if ((s = check_common(o_dtype, mode)) != EFLA_OK) return s;
     if (B < 0 || H < 0) return EFLA_ERR_SHAPE;
     if ((s = check_head(d_k, d_v)) != EFLA_OK) return s;
     const long long bh = (long long)B * H;
@@ -262,25 +279,15 @@ efla_status_t efla_decode_step(const void *q, const void *k, const void *v, efla
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(S) || !aligned16(o))
         return EFLA_ERR_ALIGN;
     const size_t xb = (size_t)bh * d_k * esize(dtype), bb = (size_t)bh * sizeof(float);
+    const size_t ob = (size_t)bh * d_v * esize(o_dtype);
     const size_t sbytes = (size_t)bh * d_k * d_v * sizeof(float);
-    if (overlaps(o, xb, q, xb) || overlaps(o, xb, k, xb) || overlaps(o, xb, v, xb) || overlaps(o, xb, beta, bb) ||
-        overlaps(o, xb, S, sbytes) || overlaps(S, sbytes, q, xb) || overlaps(S, sbytes, k, xb) ||
+    if (overlaps(o, ob, q, xb) || overlaps(o, ob, k, xb) || overlaps(o, ob, v, xb) || overlaps(o, ob, beta, bb) ||
+        overlaps(o, ob, S, sbytes) || overlaps(S, sbytes, q, xb) || overlaps(S, sbytes, k, xb) ||
         overlaps(S, sbytes, v, xb) || overlaps(S, sbytes, beta, bb))
         return EFLA_ERR_ALIAS;
     const bool eu = mode == EFLA_MODE_EULER;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (dtype == EFLA_F32) {
-        switch (d_k) {
-            case 32: return launch_decode<float, 32>(q, k, v, beta, S, o, bh, eu, st);
-            case 64: return launch_decode<float, 64>(q, k, v, beta, S, o, bh, eu, st);
-            default: return launch_decode<float, 128>(q, k, v, beta, S, o, bh, eu, st);
-        }
-    }
-    switch (d_k) {
-        case 32: return launch_decode<__nv_bfloat16, 32>(q, k, v, beta, S, o, bh, eu, st);
-        case 64: return launch_decode<__nv_bfloat16, 64>(q, k, v, beta, S, o, bh, eu, st);
-        default: return launch_decode<__nv_bfloat16, 128>(q, k, v, beta, S, o, bh, eu, st);
-    }
+    EFLA_DISPATCH(launch_decode, dtype, o_dtype, d_k, q, k, v, beta, S, o, bh, eu, st);
 }
 
 }  // extern "C"

@@ -198,9 +198,9 @@ struct StateSmem {
     __align__(16) float S[D * DVT];
 };
 
-template <typename Tin, int D>
+template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
-                                                             const float *__restrict__ S0, Tin *__restrict__ o,
+                                                             const float *__restrict__ S0, Tout *__restrict__ o,
                                                              float *__restrict__ SL, int L, int n_chunks,
                                                              SimtScratch ws) {
     extern __shared__ __align__(16) unsigned char smem_raw[];

@@ -7,7 +7,7 @@ namespace efla {
 inline bool tc_path_applies(bool bf16, int d_k, int d_v) { return false; }
 
 inline efla_status_t launch_chunk_tc(const void *, const void *, const void *, const float *, const float *, void *,
-                                     float *, long, int, bool, cudaStream_t) {
+                                     bool, float *, long, int, bool, cudaStream_t) {
     return EFLA_ERR_UNSUPPORTED;
 }
 

@@ -18,10 +18,10 @@
 
 namespace efla {
 
-template <typename T, int DK, int DV>
+template <typename T, typename To, int DK, int DV>
 __global__ void __launch_bounds__(256, 2) decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                         const T *__restrict__ v, const float *__restrict__ beta,
-                                                        float *__restrict__ S, T *__restrict__ o, bool euler) {
+                                                        float *__restrict__ S, To *__restrict__ o, bool euler) {
     constexpr int CG = DV / 4;     // column quads
     constexpr int RG = 256 / CG;   // row groups
     constexpr int RPT = DK / RG;   // rows per thread

@@ -23,10 +23,12 @@
  *      beta, alpha, lambda [B][H][L]  (fp32)
  *      S0, S_L, S          [B][H][d_k][d_v] (fp32)
  *    For decode L is absent: q,k [B][H][d_k], v,o [B][H][d_v], beta [B][H].
- *  - q, k, v and o share one storage dtype (efla_dtype_t); beta, alpha,
- *    lambda and every state are fp32.  Arithmetic is fp32 throughout (the
- *    bf16 chunk path feeds bf16 operands to tensor-core products that
- *    accumulate in fp32; the state is kept in fp32).
+ *  - q, k and v share one storage dtype (`dtype`); the output o has its
+ *    own dtype (`o_dtype`, fp32 or bf16); beta, alpha, lambda and every
+ *    state are fp32.  Arithmetic is fp32 throughout (the bf16 chunk path
+ *    feeds bf16 operands to tensor-core products that accumulate in fp32;
+ *    the state is kept in fp32).  A bf16 o adds its own rounding (up to
+ *    2^-8 relative per element) on top of the arithmetic error.
  *  - Supported head sizes: d_k == d_v in {32, 64, 128}; anything else
  *    returns EFLA_ERR_UNSUPPORTED.  B, H >= 0; L >= 0 (L = 0 copies S0 to
  *    S_L); L need not be a multiple of the internal chunk size.
@@ -122,7 +124,7 @@ size_t efla_chunk_fwd_workspace_size(efla_dtype_t dtype, int B, int H, int L,
  *   q, k  [B][H][L][d_k]   v [B][H][L][d_v]   dtype `dtype`   (inputs)
  *   beta  [B][H][L] fp32                                        (input)
  *   S0    [B][H][d_k][d_v] fp32, or NULL for the zero state     (input)
- *   o     [B][H][L][d_v] dtype `dtype`                          (output)
+ *   o     [B][H][L][d_v] dtype `o_dtype`                        (output)
  *   S_L   [B][H][d_k][d_v] fp32, or NULL if not wanted          (output)
  *   workspace / workspace_bytes: caller-owned device scratch of at least
  *     efla_chunk_fwd_workspace_size(...) bytes (may be NULL when that is 0);
@@ -133,7 +135,8 @@ size_t efla_chunk_fwd_workspace_size(efla_dtype_t dtype, int B, int H, int L,
 efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v,
                              efla_dtype_t dtype, efla_mode_t mode,
                              const float *beta, const float *S0, void *o,
-                             float *S_L, int B, int H, int L, int d_k, int d_v,
+                             efla_dtype_t o_dtype, float *S_L, int B, int H,
+                             int L, int d_k, int d_v,
                              void *workspace, size_t workspace_bytes,
                              efla_stream_t stream);
 
@@ -144,13 +147,14 @@ efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v,
  *   q, k [B][H][d_k]   v [B][H][d_v]   dtype `dtype`   (inputs)
  *   beta [B][H] fp32                                    (input)
  *   S    [B][H][d_k][d_v] fp32                          (input/output)
- *   o    [B][H][d_v] dtype `dtype`                      (output)
+ *   o    [B][H][d_v] dtype `o_dtype`                    (output)
  * o must not overlap S or any input.
  */
 efla_status_t efla_decode_step(const void *q, const void *k, const void *v,
                                efla_dtype_t dtype, efla_mode_t mode,
-                               const float *beta, float *S, void *o, int B,
-                               int H, int d_k, int d_v, efla_stream_t stream);
+                               const float *beta, float *S, void *o,
+                               efla_dtype_t o_dtype, int B, int H, int d_k,
+                               int d_v, efla_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -54,36 +54,37 @@ def test_validation_rejects_before_launch(lib):
     so, efla = lib
     F32, BF16 = 0, 1
     # bad dtype / mode
-    assert so.efla_chunk_fwd(A, A2, A3, 7, 0, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 3
-    assert so.efla_chunk_fwd(A, A2, A3, F32, 9, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 3
+    assert so.efla_chunk_fwd(A, A2, A3, 7, 0, A4, None, A5, 0, None, 1, 1, 64, 128, 128, None, 0, None) == 3
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 9, A4, None, A5, 0, None, 1, 1, 64, 128, 128, None, 0, None) == 3
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, 5, None, 1, 1, 64, 128, 128, None, 0, None) == 3
     # unsupported head sizes
-    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 48, 48, None, 0, None) == 5
-    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 128, 64, None, 0, None) == 5
-    assert so.efla_decode_step(A, A2, A3, F32, 0, A4, A5, A6, 1, 1, 256, 256, None) == 5
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, 0, None, 1, 1, 64, 48, 48, None, 0, None) == 5
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, 0, None, 1, 1, 64, 128, 64, None, 0, None) == 5
+    assert so.efla_decode_step(A, A2, A3, F32, 0, A4, A5, A6, 0, 1, 1, 256, 256, None) == 5
     # negative sizes
-    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, None, -1, 1, 64, 128, 128, None, 0, None) == 2
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, 0, None, -1, 1, 64, 128, 128, None, 0, None) == 2
     assert so.efla_gate(A, F32, 0, A2, A3, None, 1, 1, -5, 128, None) == 2
     # NULL required pointers
-    assert so.efla_chunk_fwd(None, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 1
-    assert so.efla_decode_step(A, A2, A3, BF16, 0, A4, None, A6, 1, 1, 128, 128, None) == 1
+    assert so.efla_chunk_fwd(None, A2, A3, F32, 0, A4, None, A5, 0, None, 1, 1, 64, 128, 128, None, 0, None) == 1
+    assert so.efla_decode_step(A, A2, A3, BF16, 0, A4, None, A6, 0, 1, 1, 128, 128, None) == 1
     assert so.efla_gate(None, F32, 0, A2, A3, None, 1, 1, 5, 128, None) == 1
     # misaligned pointers
     bad = ctypes.c_void_p(0x10004)
-    assert so.efla_chunk_fwd(bad, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 4
-    assert so.efla_decode_step(A, A2, A3, F32, 0, A4, bad, A6, 1, 1, 128, 128, None) == 4
+    assert so.efla_chunk_fwd(bad, A2, A3, F32, 0, A4, None, A5, 0, None, 1, 1, 64, 128, 128, None, 0, None) == 4
+    assert so.efla_decode_step(A, A2, A3, F32, 0, A4, bad, A6, 0, 1, 1, 128, 128, None) == 4
     # aliasing: o on top of q
-    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A, None, 1, 1, 64, 128, 128, None, 0, None) == 9
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A, 0, None, 1, 1, 64, 128, 128, None, 0, None) == 9
     # workspace required for the fp32 path and absent
     need = so.efla_chunk_fwd_workspace_size(F32, 1, 1, 64, 128, 128)
     assert need > 0
-    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, None, 1, 1, 64, 128, 128, None, 0, None) == 8
+    assert so.efla_chunk_fwd(A, A2, A3, F32, 0, A4, None, A5, 0, None, 1, 1, 64, 128, 128, None, 0, None) == 8
     # empty problems are accepted without any launch
-    assert so.efla_chunk_fwd(None, None, None, F32, 0, None, None, None, None, 0, 4, 64, 128, 128, None, 0,
+    assert so.efla_chunk_fwd(None, None, None, F32, 0, None, None, None, 0, None, 0, 4, 64, 128, 128, None, 0,
                              None) == 0
-    assert so.efla_decode_step(None, None, None, F32, 0, None, None, None, 3, 0, 64, 64, None) == 0
+    assert so.efla_decode_step(None, None, None, F32, 0, None, None, None, 0, 3, 0, 64, 64, None) == 0
     assert so.efla_gate(None, F32, 0, None, None, None, 2, 2, 0, 32, None) == 0
     # L = 0 without S_L: nothing to do
-    assert so.efla_chunk_fwd(None, None, None, BF16, 0, None, None, None, None, 2, 2, 0, 64, 64, None, 0,
+    assert so.efla_chunk_fwd(None, None, None, BF16, 0, None, None, None, 0, None, 2, 2, 0, 64, 64, None, 0,
                              None) == 0
 
 

@@ -28,10 +28,10 @@ def test_decode_steps_long_context_batch(efla, dtype, mode):
     Sref = np64(S)
     for s in range(steps):
         o = efla.decode_step(x["q"][s].cuda(), x["k"][s].cuda(), x["v"][s].cuda(), x["beta"][s].cuda(), Sg,
-                             mode=mode)
+                             mode=mode, out_dtype=torch.bfloat16 if s % 2 else torch.float32)
         ro, Sref = oracle.decode_step(x["q"][s], x["k"][s], x["v"][s], x["beta"][s], Sref,
                                       euler=(mode == "euler"))
-        assert_close(o, ro, dtype, f"o step {s}")
+        assert_close(o, ro, dtype, f"o step {s}", out_bf16=bool(s % 2))
     torch.cuda.synchronize()
     # the state is fp32 in both arms: hold it to the fp32 bar
     assert_close(Sg, Sref, "f32", "S")
