@@ -43,22 +43,6 @@ efla_status_t check_head(int d_k, int d_v) {
 
 efla_status_t launched() { return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA; }
 
-// Opt a kernel into more than 48 KB of dynamic shared memory once per
-// device.  Later calls (including ones made while a stream is being
-// captured into a CUDA graph) skip the runtime call.
-template <auto Kernel>
-bool ensure_smem(size_t bytes) {
-    static std::atomic<uint64_t> done{0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    const uint64_t bit = 1ull << (dev & 63);
-    if (done.load(std::memory_order_acquire) & bit) return true;
-    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
-        return false;
-    done.fetch_or(bit, std::memory_order_acq_rel);
-    return true;
-}
-
 int num_sms() {
     static std::atomic<int> cached[64];
     int dev = 0, n = 0;

@@ -1,14 +1,677 @@
-// efla_chunk_tc.cuh - tensor-core (tcgen05) chunked prefill for bf16 inputs.
+// efla_chunk_tc.cuh - fused chunked prefill on the 5th-generation tensor
+// cores (tcgen05 + TMEM + TMA) for bf16 q/k/v, d_k = d_v = 128.
+//
+// Computes the recurrence of "Exact Flow Linear Attention" (papernotes.org
+// summary of arXiv 2512.12602, 关键设计 2; readout of the 整体框架
+// flowchart) chunk by chunk in the UT form of the chunk-parallel scheme that
+// page cites (整体框架, "WY / UT"), with C = 64:
+//
+//   alpha = gate(beta, ||k||^2)                       (fp32, CUDA cores)
+//   G  = [K; Q] K^T                                   (tcgen05, M=128 N=64 K=128)
+//   A  = strictly-lower(diag(alpha) K K^T);  T = (I + A)^{-1}   (fp32, CUDA cores)
+//   X  = [0; T diag(alpha)]                           (bf16 hi + lo operands)
+//   [. ; W] = X K,   [0; U] = X V_tile                (tcgen05, N=128 and N=64)
+//   Y += [Q; -W] S  ->  [Q S; U - W S] = [Q S; D]     (tcgen05, N=64 K=128)
+//   S += K^T D                                        (tcgen05, N=64 K=64)
+//   Y += [M; *] D   ->  O = Q S + M D,  M = lower-incl-diag(Q K^T)
+//
+// Every product is stacked to M = 128 rows so the accumulator of each
+// tcgen05.mma occupies all 128 TMEM lanes, one row per lane.  (In the last
+// product the lower 64 rows of the A operand are whatever follows M in shared
+// memory: they only add into the D rows of Y, which are dead by then.)
+//
+// Precision: q, k, v are exact bf16 operands.  T diag(alpha), S, D and M are
+// fp32 values fed to the bf16 tensor cores as a hi + lo pair of bf16
+// (x = hi + lo to ~16 significant bits); only -W goes in as a single bf16.
+// Accumulation is fp32 in TMEM and the state is kept in fp32.
+//
+// One CTA per (b, h, half of d_v): the 128 x 64 fp32 state tile lives in
+// TMEM for the whole sequence.  Warp roles:
+//   warps 0-3  "prep":  gate, T, X and -W for chunk n+1 (S-independent)
+//   warps 4-7  "state": D -> bf16, S -> bf16 and O -> HBM for chunk n
+//   warp 8     one thread issues every tcgen05.mma and commit
+//   warp 9     one thread issues the TMA loads (2-stage K/Q/V ring)
+// Every mbarrier wait is bounded; a wait that gives up sets the sticky
+// device error word and an abort flag, every role then leaves its loop, the
+// MMA thread drains its outstanding MMAs and the TMA thread its copies, and
+// the CTA frees its TMEM before returning.
 #pragma once
+#include <cuda.h>
+
+#include <mutex>
+
+#include "../../include/efla.h"
 #include "efla_common.cuh"
+#include "efla_tc_ptx.cuh"
 
 namespace efla {
+namespace tc {
 
-inline bool tc_path_applies(bool bf16, int d_k, int d_v) { return false; }
+constexpr int C = 64, DK = 128, DVT = 64, NSPLIT = 2;
+constexpr int kThreads = 320;
+constexpr uint32_t SLOT = 8192;                 // one 64 x 64 bf16 swizzled box
+constexpr uint32_t STAGE = 7 * SLOT;            // K0 Q0 W0 K1 Q1 W1 V
+constexpr uint32_t SL_K0 = 0, SL_Q0 = 1, SL_W0 = 2, SL_V = 6;
+constexpr uint32_t BOXSTRIDE = 3 * SLOT;        // K0->K1, Q0->Q1, W0->W1
+constexpr int LDF = 64;                         // fp32 row stride of A and T
+constexpr uint32_t OFF_M = 2 * STAGE;           // M hi/lo for chunk parity 0 and 1: 4 boxes
+constexpr uint32_t OFF_Z0 = OFF_M + 4 * SLOT;   // zero box, then T' hi  ([0; T'hi] operand)
+constexpr uint32_t OFF_THI = OFF_Z0 + SLOT;
+constexpr uint32_t OFF_Z1 = OFF_THI + SLOT;     // zero box, then T' lo  ([0; T'lo] operand)
+constexpr uint32_t OFF_TLO = OFF_Z1 + SLOT;
+constexpr uint32_t OFF_SB = OFF_TLO + SLOT;     // S tile bf16 hi, then lo (MN-major B), 128 x 64 each
+constexpr uint32_t OFF_DB = OFF_SB + 4 * SLOT;  // D bf16 hi, then lo (MN-major B), 64 x 64 each
+constexpr uint32_t OFF_ALPHA = OFF_DB + 2 * SLOT;
+constexpr uint32_t OFF_BAR = OFF_ALPHA + 256;
+constexpr uint32_t NBAR = 16;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+// fp32 scratch of the T computation aliases buffers that are idle meanwhile:
+// A (64 x 64) the two W boxes of the stage being prepared (rows 0-31 / 32-63),
+// T (64 x 64) the T' hi / lo boxes (rows 0-31 / 32-63).
 
-inline efla_status_t launch_chunk_tc(const void *, const void *, const void *, const float *, const float *, void *,
-                                     bool, float *, long, int, bool, cudaStream_t) {
-    return EFLA_ERR_UNSUPPORTED;
+// TMEM columns (fp32, 128 lanes)
+constexpr uint32_t T_S = 0, T_G = 64, T_YW = 128, T_YU = 256, TMEM_COLS = 512;
+
+enum : int {
+    B_FULL = 0,     // [2] TMA stage landed
+    B_EMPTY = 2,    // [2] stage free again (commit after the last MMA reading it)
+    B_GFULL = 4,    // G ready in TMEM
+    B_GEMPTY = 5,   // prep has read G
+    B_XFULL = 6,    // X written
+    B_YFULL = 7,    // X K and X V done
+    B_A2FULL = 8,   // [2] -W and M written for chunk parity b
+    B_SBFULL = 10,  // bf16 S tile written
+    B_DFULL = 11,   // Y += [Q;-W] S done
+    B_DELTA = 12,   // bf16 D written
+    B_SFULL = 13,   // S += K^T D and O += M D done
+    B_DRAIN = 14,   // final drain of the MMA pipe
+};
+
+constexpr uint32_t ID_G = ptx::idesc_bf16(128, 64, false, false);
+constexpr uint32_t ID_YW = ptx::idesc_bf16(128, 128, false, true);
+constexpr uint32_t ID_N64 = ptx::idesc_bf16(128, 64, false, true);
+constexpr uint32_t ID_S = ptx::idesc_bf16(128, 64, true, true);
+
+__device__ __forceinline__ bool bar_any(uint32_t id, uint32_t n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+// Row r of a 64 x 64 fp32 matrix stored as two 32-row halves.
+struct Split64 {
+    float *lo, *hi;
+    __device__ __forceinline__ float *row(int r) const { return (r < 32 ? lo : hi) + (r & 31) * LDF; }
+};
+
+// T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A, by 16 x 16
+// diagonal blocks (right-looking forward substitution, one warp per block)
+// followed by three block rows  T_I,<I = -T_II (A_I,<I T_<I,<I).  Row block I
+// of A is overwritten by the intermediate product.  128 threads (prep).
+__device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af, const Split64 Tf) {
+    {
+        const int w = p >> 5, l = p & 31, c = l & 15, h = l >> 4, base = 16 * w;
+        float acc[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) acc[s] = (2 * s + h == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const float x = __shfl_sync(0xffffffffu, acc[m >> 1], ((m & 1) << 4) | c);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) acc[s] = fmaf(-Af.row(base + 2 * s + h)[base + m], x, acc[s]);
+        }
+#pragma unroll
+        for (int s = 0; s < 8; ++s) Tf.row(base + 2 * s + h)[base + c] = acc[s];
+    }
+    ptx::named_bar(1, 128);
+#pragma unroll 1
+    for (int I = 1; I < 4; ++I) {
+        const int W = 16 * I, nent = 16 * W;
+        float R[6];
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+            const int e = p + 128 * k;
+            float acc = 0.f;
+            if (e < nent) {
+                const int i = e / W, j = e % W;
+                const float *arow = Af.row(16 * I + i);
+                for (int m = (j & ~15); m < W; ++m) acc = fmaf(arow[m], Tf.row(m)[j], acc);
+            }
+            R[k] = acc;
+        }
+        ptx::named_bar(1, 128);
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+            const int e = p + 128 * k;
+            if (e < nent) Af.row(16 * I + e / W)[e % W] = R[k];
+        }
+        ptx::named_bar(1, 128);
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+            const int e = p + 128 * k;
+            if (e < nent) {
+                const int i = e / W, j = e % W;
+                const float *trow = Tf.row(16 * I + i) + 16 * I;
+                float acc = 0.f;
+                for (int m = 0; m <= i; ++m) acc = fmaf(trow[m], Af.row(16 * I + m)[j], acc);
+                Tf.row(16 * I + i)[j] = -acc;
+            }
+        }
+        ptx::named_bar(1, 128);
+    }
+}
+
+// bf16 hi + lo split of a pair of fp32 values (hi = rn(x), lo = rn(x - hi)).
+// One 64-value fp32 row (held as two 32-register halves) -> bf16 hi at
+// `base` and lo at `base + lo_off`, row `row` of a 128-byte-swizzled tile.
+__device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo_off, int row, const uint32_t (&a)[32],
+                                                const uint32_t (&b)[32]);
+
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+    hi = ptx::pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
+    lo = ptx::pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+}
+
+__device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo_off, int row, const uint32_t (&a)[32],
+                                                const uint32_t (&b)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint32_t h4[4], l4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c0 = 8 * j + 2 * u;
+            const float x0 = __uint_as_float(c0 < 32 ? a[c0] : b[c0 - 32]);
+            const float x1 = __uint_as_float(c0 + 1 < 32 ? a[c0 + 1] : b[c0 + 1 - 32]);
+            split2(x0, x1, h4[u], l4[u]);
+        }
+        *reinterpret_cast<uint4 *>(base + ptx::sw128_chunk(row, j)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+        *reinterpret_cast<uint4 *>(base + lo_off + ptx::sw128_chunk(row, j)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+    }
+}
+
+template <typename Tout>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ beta,
+                    const float *__restrict__ S0, Tout *__restrict__ o, float *__restrict__ SL, int L, int nc,
+                    int euler) {
+    using namespace ptx;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 4);
+    float *alpha_s = reinterpret_cast<float *>(sm + OFF_ALPHA);
+    const Split64 Tf{reinterpret_cast<float *>(sm + OFF_THI), reinterpret_cast<float *>(sm + OFF_TLO)};
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long bh = blockIdx.x / NSPLIT;
+    const int j0 = (blockIdx.x % NSPLIT) * DVT;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(&bar[B_FULL], 1);
+        mbar_init(&bar[B_FULL + 1], 1);
+        mbar_init(&bar[B_EMPTY], 1);
+        mbar_init(&bar[B_EMPTY + 1], 1);
+        mbar_init(&bar[B_GFULL], 1);
+        mbar_init(&bar[B_GEMPTY], 128);
+        mbar_init(&bar[B_XFULL], 128);
+        mbar_init(&bar[B_YFULL], 1);
+        mbar_init(&bar[B_A2FULL], 128);
+        mbar_init(&bar[B_A2FULL + 1], 128);
+        mbar_init(&bar[B_SBFULL], 128);
+        mbar_init(&bar[B_DFULL], 1);
+        mbar_init(&bar[B_DELTA], 128);
+        mbar_init(&bar[B_SFULL], 1);
+        mbar_init(&bar[B_DRAIN], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    // constant zero boxes: rows 0-63 of the [0; T' hi] and [0; T' lo] operands
+    for (int i = threadIdx.x; i < 2 * (int)SLOT / 16; i += kThreads) {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(sm + (i < (int)SLOT / 16 ? OFF_Z0 : OFF_Z1 - SLOT) + 16 * i) = z;
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ prep
+        const int p = threadIdx.x;
+        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+        for (int n = 0; n < nc; ++n) {
+            const int s = n & 1;
+            unsigned char *st = sm + s * STAGE;
+            const int t0 = n * C;
+            bool ok = mbar_wait(&bar[B_FULL + s], (n >> 1) & 1, abort_flag);
+            if (bar_any(1, 128, !ok || *abort_flag)) break;
+            {   // gate: two lanes per key row, each over one 64-wide half
+                const int r = p >> 1, h = p & 1;
+                const unsigned char *krow = st + (h ? BOXSTRIDE : 0) + SL_K0 * SLOT + r * 128;
+                float ss = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float f[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(krow + 16 * j), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                if (h == 0) {
+                    const int t = t0 + r;
+                    alpha_s[r] = (t < L) ? gate_alpha(beta[bh * (long)L + t], ss, euler != 0) : 0.f;
+                }
+            }
+            named_bar(1, 128);
+            ok = mbar_wait(&bar[B_GFULL], n & 1, abort_flag);
+            if (bar_any(1, 128, !ok || *abort_flag)) break;
+            tc_fence_after();
+            uint32_t ga[32], gb[32];
+            tmem_ld32(tl + T_G, ga);
+            tmem_ld32(tl + T_G + 32, gb);
+            tmem_ld_wait(ga);
+            tmem_ld_wait(gb);
+            tc_fence_before();
+            mbar_arrive(&bar[B_GEMPTY]);
+            const Split64 Af{reinterpret_cast<float *>(st + SL_W0 * SLOT),
+                             reinterpret_cast<float *>(st + SL_W0 * SLOT + BOXSTRIDE)};
+            if (p < 64) {  // A row p = alpha_p * (K K^T)[p][c] for c < p
+                const float ap = alpha_s[p];
+                float *arow = Af.row(p);
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    float4 v;
+                    float *vv = reinterpret_cast<float *>(&v);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t bits = (c + e < 32) ? ga[c + e] : gb[c + e - 32];
+                        vv[e] = (c + e < p) ? ap * __uint_as_float(bits) : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(arow + c) = v;
+                }
+            } else {       // M row r = (Q K^T)[r][c] for c <= r, as bf16 hi and lo boxes
+                const int r = p - 64;
+                unsigned char *mhi = sm + OFF_M + (n & 1) * 2 * SLOT, *mlo = mhi + SLOT;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t h4[4], l4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c0 = 8 * j + 2 * e;
+                        const float x0 = (c0 <= r) ? __uint_as_float(c0 < 32 ? ga[c0] : gb[c0 - 32]) : 0.f;
+                        const float x1 =
+                            (c0 + 1 <= r) ? __uint_as_float(c0 + 1 < 32 ? ga[c0 + 1] : gb[c0 + 1 - 32]) : 0.f;
+                        split2(x0, x1, h4[e], l4[e]);
+                    }
+                    *reinterpret_cast<uint4 *>(mhi + sw128_chunk(r, j)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+                    *reinterpret_cast<uint4 *>(mlo + sw128_chunk(r, j)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+                }
+            }
+            named_bar(1, 128);
+            invert_unit_lower(p, Af, Tf);
+            // T' = T diag(alpha) as bf16 hi/lo into the boxes T itself occupies:
+            // gather this thread's 32 values first, then overwrite.
+            uint32_t th[16], tlo[16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = p + 128 * i, r = e >> 3, j = e & 7;
+                const float *trow = Tf.row(r);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c0 = 8 * j + 2 * u;
+                    const float x0 = (c0 <= r) ? trow[c0] * alpha_s[c0] : 0.f;
+                    const float x1 = (c0 + 1 <= r) ? trow[c0 + 1] * alpha_s[c0 + 1] : 0.f;
+                    split2(x0, x1, th[4 * i + u], tlo[4 * i + u]);
+                }
+            }
+            named_bar(1, 128);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = p + 128 * i, r = e >> 3, j = e & 7;
+                *reinterpret_cast<uint4 *>(sm + OFF_THI + sw128_chunk(r, j)) =
+                    make_uint4(th[4 * i], th[4 * i + 1], th[4 * i + 2], th[4 * i + 3]);
+                *reinterpret_cast<uint4 *>(sm + OFF_TLO + sw128_chunk(r, j)) =
+                    make_uint4(tlo[4 * i], tlo[4 * i + 1], tlo[4 * i + 2], tlo[4 * i + 3]);
+            }
+            fence_proxy_async();
+            mbar_arrive(&bar[B_XFULL]);
+            ok = mbar_wait(&bar[B_YFULL], n & 1, abort_flag);
+            if (bar_any(1, 128, !ok || *abort_flag)) break;
+            tc_fence_after();
+            if (warp >= 2) {  // W rows live in TMEM lanes 64..127: write -W into the stage
+                const int r = p - 64;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t wa[32], wb[32];
+                    tmem_ld32(tl + T_YW + 64 * h, wa);
+                    tmem_ld32(tl + T_YW + 64 * h + 32, wb);
+                    tmem_ld_wait(wa);
+                    tmem_ld_wait(wb);
+                    unsigned char *wrow = st + SL_W0 * SLOT + h * BOXSTRIDE;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int c0 = 8 * j + 2 * u;
+                            const float x0 = __uint_as_float(c0 < 32 ? wa[c0] : wb[c0 - 32]);
+                            const float x1 = __uint_as_float(c0 + 1 < 32 ? wa[c0 + 1] : wb[c0 + 1 - 32]);
+                            w4[u] = pack_bf16(-x0, -x1);
+                        }
+                        *reinterpret_cast<uint4 *>(wrow + sw128_chunk(r, j)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(&bar[B_A2FULL + (n & 1)]);
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ state
+        const int q = threadIdx.x - 128;  // TMEM lane / state row
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        {
+            uint32_t ra[32], rb[32];
+            const float *src = S0 ? S0 + ((size_t)bh * DK + q) * DK + j0 : nullptr;
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+                const float4 v = src ? *reinterpret_cast<const float4 *>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                uint32_t *dst = (c < 32) ? &ra[c] : &rb[c - 32];
+                dst[0] = __float_as_uint(v.x);
+                dst[1] = __float_as_uint(v.y);
+                dst[2] = __float_as_uint(v.z);
+                dst[3] = __float_as_uint(v.w);
+            }
+            tmem_st32(tl + T_S, ra);
+            tmem_st32(tl + T_S + 32, rb);
+            tmem_st_wait();
+            write_split_row(sm + OFF_SB, 2 * SLOT, q, ra, rb);
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(&bar[B_SBFULL]);
+        }
+        for (int n = 0; n < nc; ++n) {
+            const int b = n & 1;
+            const int t0 = n * C;
+            bool ok = mbar_wait(&bar[B_DFULL], n & 1, abort_flag);
+            if (bar_any(2, 128, !ok || *abort_flag)) break;
+            tc_fence_after();
+            if (warp >= 6) {  // D rows (lanes 64..127) -> bf16 MN-major operand, row c = lane - 64
+                const int c = q - 64;
+                uint32_t da[32], db[32];
+                tmem_ld32(tl + T_YU + 64 * b, da);
+                tmem_ld32(tl + T_YU + 64 * b + 32, db);
+                tmem_ld_wait(da);
+                tmem_ld_wait(db);
+                write_split_row(sm + OFF_DB, SLOT, c, da, db);
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(&bar[B_DELTA]);
+            ok = mbar_wait(&bar[B_SFULL], n & 1, abort_flag);
+            if (bar_any(2, 128, !ok || *abort_flag)) break;
+            tc_fence_after();
+            uint32_t sa[32], sb[32];
+            tmem_ld32(tl + T_S, sa);
+            tmem_ld32(tl + T_S + 32, sb);
+            tmem_ld_wait(sa);
+            tmem_ld_wait(sb);
+            write_split_row(sm + OFF_SB, 2 * SLOT, q, sa, sb);
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(&bar[B_SBFULL]);
+            if (warp < 6) {  // O rows (lanes 0..63)
+                uint32_t oa[32], ob[32];
+                tmem_ld32(tl + T_YU + 64 * b, oa);
+                tmem_ld32(tl + T_YU + 64 * b + 32, ob);
+                tmem_ld_wait(oa);
+                tmem_ld_wait(ob);
+                if (t0 + q < L) {
+                    Tout *dst = o + ((size_t)bh * L + t0 + q) * DK + j0;
+#pragma unroll
+                    for (int c = 0; c < 64; c += 4) {
+                        const uint32_t *src = (c < 32) ? &oa[c] : &ob[c - 32];
+                        store4(dst + c, make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
+                                                    __uint_as_float(src[2]), __uint_as_float(src[3])));
+                    }
+                }
+            }
+            if (n == nc - 1 && SL) {
+                float *dst = SL + ((size_t)bh * DK + q) * DK + j0;
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    const uint32_t *src = (c < 32) ? &sa[c] : &sb[c - 32];
+                    *reinterpret_cast<float4 *>(dst + c) = make_float4(
+                        __uint_as_float(src[0]), __uint_as_float(src[1]), __uint_as_float(src[2]),
+                        __uint_as_float(src[3]));
+                }
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t sba = sbase + OFF_SB, dba = sbase + OFF_DB;
+            const uint32_t xhi = sbase + OFF_Z0, xlo = sbase + OFF_Z1;  // [0; T' hi], [0; T' lo]
+            auto stage_addr = [&](int n) { return sbase + (uint32_t)(n & 1) * STAGE; };
+            auto issue_G = [&](int n) {
+                const uint32_t sa = stage_addr(n);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a = sa + SL_K0 * SLOT + (kk >> 2) * BOXSTRIDE + (kk & 3) * 32;
+                    mma_bf16(tmem + T_G, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), ID_G, kk > 0);
+                }
+                mma_commit(&bar[B_GFULL]);
+            };
+            auto issue_Y = [&](int n) {  // Y = X_hi [K | V] + X_lo [K | V]
+                const uint32_t sa = stage_addr(n), yu = tmem + T_YU + 64 * (n & 1);
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t xa = part ? xlo : xhi;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + T_YW, sdesc_sw128(xa + kk * 32, 16, 1024),
+                                 sdesc_sw128(sa + SL_K0 * SLOT + kk * 2048, BOXSTRIDE, 1024), ID_YW, part | kk);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(yu, sdesc_sw128(xa + kk * 32, 16, 1024),
+                                 sdesc_sw128(sa + SL_V * SLOT + kk * 2048, SLOT, 1024), ID_N64, part | kk);
+                }
+                mma_commit(&bar[B_YFULL]);
+            };
+            auto issue_D = [&](int n) {  // Y += [Q; -W] (S_hi + S_lo)
+                const uint32_t sa = stage_addr(n), yu = tmem + T_YU + 64 * (n & 1);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t a = sa + SL_Q0 * SLOT + (kk >> 2) * BOXSTRIDE + (kk & 3) * 32;
+                        mma_bf16(yu, sdesc_sw128(a, 16, 1024),
+                                 sdesc_sw128(sba + part * 2 * SLOT + kk * 2048, SLOT, 1024), ID_N64, 1);
+                    }
+                mma_commit(&bar[B_DFULL]);
+            };
+            auto issue_SO = [&](int n) {  // S += K^T (D_hi + D_lo);  Y += M_hi D_hi + M_hi D_lo + M_lo D_hi
+                const uint32_t sa = stage_addr(n), yu = tmem + T_YU + 64 * (n & 1);
+                const uint32_t mhi = sbase + OFF_M + (n & 1) * 2 * SLOT, mlo = mhi + SLOT;
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + T_S, sdesc_sw128(sa + SL_K0 * SLOT + kk * 2048, BOXSTRIDE, 1024),
+                                 sdesc_sw128(dba + part * SLOT + kk * 2048, SLOT, 1024), ID_S, 1);
+#pragma unroll
+                for (int part = 0; part < 3; ++part) {
+                    const uint32_t ma = (part == 2) ? mlo : mhi, da = dba + (part == 1 ? SLOT : 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(yu, sdesc_sw128(ma + kk * 32, 16, 1024), sdesc_sw128(da + kk * 2048, SLOT, 1024),
+                                 ID_N64, 1);
+                }
+                mma_commit(&bar[B_SFULL]);
+                mma_commit(&bar[B_EMPTY + (n & 1)]);
+            };
+            bool ok = true;
+            do {
+                if (!(ok = mbar_wait(&bar[B_FULL], 0, abort_flag))) break;
+                tc_fence_after();
+                issue_G(0);
+                if (!(ok = mbar_wait(&bar[B_XFULL], 0, abort_flag))) break;
+                tc_fence_after();
+                issue_Y(0);
+                if (nc > 1) {
+                    if (!(ok = mbar_wait(&bar[B_FULL + 1], 0, abort_flag))) break;
+                    if (!(ok = mbar_wait(&bar[B_GEMPTY], 0, abort_flag))) break;
+                    tc_fence_after();
+                    issue_G(1);
+                }
+                for (int n = 0; n < nc; ++n) {
+                    if (!(ok = mbar_wait(&bar[B_A2FULL + (n & 1)], (n >> 1) & 1, abort_flag))) break;
+                    if (!(ok = mbar_wait(&bar[B_SBFULL], n & 1, abort_flag))) break;
+                    tc_fence_after();
+                    issue_D(n);
+                    if (!(ok = mbar_wait(&bar[B_DELTA], n & 1, abort_flag))) break;
+                    tc_fence_after();
+                    issue_SO(n);
+                    if (n + 1 < nc) {
+                        if (!(ok = mbar_wait(&bar[B_XFULL], (n + 1) & 1, abort_flag))) break;
+                        tc_fence_after();
+                        issue_Y(n + 1);
+                    }
+                    if (n + 2 < nc) {
+                        if (!(ok = mbar_wait(&bar[B_FULL + (n & 1)], ((n + 2) >> 1) & 1, abort_flag))) break;
+                        if (!(ok = mbar_wait(&bar[B_GEMPTY], (n + 1) & 1, abort_flag))) break;
+                        tc_fence_after();
+                        issue_G(n + 2);
+                    }
+                }
+            } while (0);
+            // drain: wait (bounded, even after an abort) until every MMA issued has completed
+            mma_commit(&bar[B_DRAIN]);
+            int never = 0;
+            mbar_wait(&bar[B_DRAIN], 0, &never);
+        }
+    } else {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch(&tm_q);
+            tma_prefetch(&tm_k);
+            tma_prefetch(&tm_v);
+            int last[2] = {-1, -1};
+            for (int n = 0; n < nc; ++n) {
+                const int s = n & 1;
+                if (n >= 2 && !mbar_wait(&bar[B_EMPTY + s], ((n >> 1) - 1) & 1, abort_flag)) break;
+                if (*abort_flag) break;
+                unsigned char *st = sm + s * STAGE;
+                uint64_t *fb = &bar[B_FULL + s];
+                mbar_expect_tx(fb, 5 * SLOT);
+                const int y = n * C, z = (int)bh;
+                tma_load_3d(st + SL_K0 * SLOT, &tm_k, fb, 0, y, z);
+                tma_load_3d(st + SL_K0 * SLOT + BOXSTRIDE, &tm_k, fb, 64, y, z);
+                tma_load_3d(st + SL_Q0 * SLOT, &tm_q, fb, 0, y, z);
+                tma_load_3d(st + SL_Q0 * SLOT + BOXSTRIDE, &tm_q, fb, 64, y, z);
+                tma_load_3d(st + SL_V * SLOT, &tm_v, fb, j0, y, z);
+                last[s] = n;
+            }
+            // drain: every copy this thread started has landed before the CTA exits
+            int never = 0;
+            for (int s = 0; s < 2; ++s)
+                if (last[s] >= 0) mbar_wait(&bar[B_FULL + s], (last[s] >> 1) & 1, &never);
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D view [bh][L][128] of a bf16 [B][H][L][128] tensor, 64 x 64 boxes,
+// 128-byte swizzle; rows past L read as zero.
+inline bool make_map(CUtensorMap *m, const void *base, long bh, int L) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)L, (cuuint64_t)bh};
+    const cuuint64_t strides[2] = {(cuuint64_t)DK * 2, (cuuint64_t)L * DK * 2};
+    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename Tout>
+inline efla_status_t launch(const void *q, const void *k, const void *v, const float *beta, const float *S0,
+                            void *o, float *SL, long bh, int L, bool euler, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, bh, L) || !make_map(&mk, k, bh, L) || !make_map(&mv, v, bh, L)) return EFLA_ERR_CUDA;
+    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES)) return EFLA_ERR_CUDA;
+    const long grid = bh * NSPLIT;
+    if (grid > 0x7fffffffL) return EFLA_ERR_SHAPE;
+    const int nc = (L + C - 1) / C;
+    chunk_tc_kernel<Tout><<<(unsigned)grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mv, beta, S0, static_cast<Tout *>(o),
+                                                                         SL, L, nc, euler ? 1 : 0);
+    return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
+}
+
+}  // namespace tc
+
+// The tensor-core kernel takes bf16 q/k/v with d_k = d_v = 128.
+inline bool tc_path_applies(bool bf16, int d_k, int d_v) { return bf16 && d_k == 128 && d_v == 128; }
+
+inline efla_status_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *beta,
+                                     const float *S0, void *o, bool o_bf16, float *SL, long bh, int L, bool euler,
+                                     cudaStream_t st) {
+    return o_bf16 ? tc::launch<__nv_bfloat16>(q, k, v, beta, S0, o, SL, bh, L, euler, st)
+                  : tc::launch<float>(q, k, v, beta, S0, o, SL, bh, L, euler, st);
 }
 
 }  // namespace efla

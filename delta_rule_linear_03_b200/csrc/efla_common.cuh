@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace efla {
 
 // Sticky device error word: a kernel whose bounded wait gives up ORs a
@@ -63,6 +65,22 @@ __device__ __forceinline__ float warp_sum(float x, unsigned mask = 0xffffffffu) 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(mask, x, o);
     return x;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory once per
+// device.  Later calls (including ones made while a stream is being
+// captured into a CUDA graph) skip the runtime call.
+template <auto Kernel>
+inline bool ensure_smem(size_t bytes) {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return false;
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return true;
 }
 
 }  // namespace efla
