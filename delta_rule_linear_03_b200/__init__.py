@@ -40,7 +40,9 @@ STATUS = {0: "EFLA_OK", 1: "EFLA_ERR_NULL", 2: "EFLA_ERR_SHAPE", 3: "EFLA_ERR_DT
           5: "EFLA_ERR_UNSUPPORTED", 6: "EFLA_ERR_CUDA", 7: "EFLA_ERR_TIMEOUT", 8: "EFLA_ERR_WORKSPACE",
           9: "EFLA_ERR_ALIAS"}
 EXPORTS = ("efla_status_string", "efla_version", "efla_last_error", "efla_gate",
-           "efla_chunk_fwd_workspace_size", "efla_chunk_fwd", "efla_decode_step")
+           "efla_chunk_fwd_workspace_size", "efla_chunk_fwd", "efla_decode_step",
+           "efla_chunk_fwd_workspace_size_simt", "efla_chunk_fwd_noalloc")
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _p, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 _lib.efla_status_string.restype = ctypes.c_char_p
@@ -55,6 +57,10 @@ _lib.efla_chunk_fwd_workspace_size.restype = _sz
 _lib.efla_chunk_fwd_workspace_size.argtypes = [_i, _i, _i, _i, _i, _i]
 _lib.efla_chunk_fwd.restype = _i
 _lib.efla_chunk_fwd.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _p, _sz, _p]
+_lib.efla_chunk_fwd_workspace_size_simt.restype = _sz
+_lib.efla_chunk_fwd_workspace_size_simt.argtypes = [_i, _i, _i, _i, _i]
+_lib.efla_chunk_fwd_noalloc.restype = _i
+_lib.efla_chunk_fwd_noalloc.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _p]
 _lib.efla_decode_step.restype = _i
 _lib.efla_decode_step.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 
@@ -162,6 +168,31 @@ def chunk_fwd(q, k, v, beta, S0=None, mode: str = "exact", o=None, S_L=None, wan
                                    _ptr(o), _dt(o), _ptr(S_L), B, H, L, dk, dv,
                                    _ptr(workspace) if need else None, wbytes if need else 0,
                                    _stream(dev)), "efla_chunk_fwd")
+    return o, S_L
+
+
+def chunk_fwd_noalloc(q, k, v, beta, S0=None, mode: str = "exact", o=None, S_L=None,
+                      want_state: bool = True, out_dtype=torch.float32):
+    """``chunk_fwd`` through the entry point that allocates no device memory
+    (its scratch is a fixed 32 MiB array inside the library, shared by all
+    calls on a device; calls that overlap on the GPU race on it).  For hosts
+    that cannot let a library allocate.  Outputs are allocated here only when
+    not passed in."""
+    dev = _dev(q, k, v, beta, S0)
+    B, H, L, dk = k.shape
+    dv = v.shape[-1]
+    if q.shape != k.shape or v.shape[:3] != (B, H, L) or q.dtype != k.dtype or v.dtype != k.dtype:
+        raise ValueError("q, k, v must share dtype and [B,H,L,*] shape")
+    if beta.dtype != torch.float32 or tuple(beta.shape) != (B, H, L):
+        raise ValueError("beta must be float32 [B,H,L]")
+    o = torch.empty((B, H, L, dv), dtype=out_dtype, device=dev) if o is None else o
+    if want_state and S_L is None:
+        S_L = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _dev(o, S_L)
+    with torch.cuda.device(dev):
+        _check(_lib.efla_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _dt(q), MODES[mode], _ptr(beta),
+                                           _ptr(S0), _ptr(o), _dt(o), _ptr(S_L), B, H, L, dk, dv,
+                                           _stream(dev)), "efla_chunk_fwd_noalloc")
     return o, S_L
 
 

@@ -275,3 +275,79 @@ efla_status_t efla_decode_step(const void *q, const void *k, const void *v, efla
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation variant of the chunked prefill.
+//
+// For callers that cannot allocate device memory (an engine that owns every
+// byte of GPU memory through its own pool, or a loop where cudaMalloc's
+// implicit synchronisation is not acceptable): the CUDA-core chunked kernels
+// run with their scratch in this fixed file-scope array instead of a
+// caller-provided workspace.  Every GPU that loads the library holds it
+// until the process exits; all calls on a device share it.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[EFLA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device.  Host code must not use the symbol itself as a pointer: on the
+// host it is only a stand-in for the device variable.
+void *noalloc_scratch_ptr() {
+    static std::atomic<uintptr_t> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    uintptr_t p = cached[dev].load(std::memory_order_acquire);
+    if (p) return reinterpret_cast<void *>(p);
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return nullptr;
+    cached[dev].store(reinterpret_cast<uintptr_t>(addr), std::memory_order_release);
+    return addr;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t efla_chunk_fwd_workspace_size_simt(int B, int H, int L, int d_k, int d_v) {
+    if (B <= 0 || H <= 0 || L <= 0 || check_head(d_k, d_v) != EFLA_OK) return 0;
+    return simt_workspace_bytes((long)B * H, L, d_k);
+}
+
+efla_status_t efla_chunk_fwd_noalloc(const void *q, const void *k, const void *v, efla_dtype_t dtype,
+                                     efla_mode_t mode, const float *beta, const float *S0, void *o,
+                                     efla_dtype_t o_dtype, float *S_L, int B, int H, int L, int d_k, int d_v,
+                                     efla_stream_t stream) {
+    efla_status_t s = check_common(dtype, mode);
+    if (s != EFLA_OK) return s;
+    if ((s = check_common(o_dtype, mode)) != EFLA_OK) return s;
+    if (B < 0 || H < 0 || L < 0) return EFLA_ERR_SHAPE;
+    if ((s = check_head(d_k, d_v)) != EFLA_OK) return s;
+    const long long bh = (long long)B * H;
+    if (bh * (long long)(L > 0 ? L : 1) * d_k > kMaxElems || bh > 0x7fffffffLL) return EFLA_ERR_SHAPE;
+    if (bh == 0 || L == 0)  // nothing uses scratch: the regular entry point handles these allocation-free
+        return efla_chunk_fwd(q, k, v, dtype, mode, beta, S0, o, o_dtype, S_L, B, H, L, d_k, d_v, nullptr, 0,
+                              stream);
+    const size_t need = simt_workspace_bytes(bh, L, d_k);
+    if (need > EFLA_NOALLOC_SCRATCH_BYTES) return EFLA_ERR_WORKSPACE;
+    if (!q || !k || !v || !beta || !o) return EFLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(beta) || !aligned16(o) ||
+        (S0 && !aligned16(S0)) || (S_L && !aligned16(S_L)))
+        return EFLA_ERR_ALIGN;
+    const size_t xb = (size_t)bh * L * d_k * esize(dtype), bb = (size_t)bh * L * sizeof(float);
+    const size_t ob = (size_t)bh * L * d_v * esize(o_dtype);
+    const size_t sbytes = (size_t)bh * d_k * d_v * sizeof(float);
+    if (overlaps(o, ob, q, xb) || overlaps(o, ob, k, xb) || overlaps(o, ob, v, xb) || overlaps(o, ob, beta, bb) ||
+        overlaps(o, ob, S0, sbytes))
+        return EFLA_ERR_ALIAS;
+    if (S_L && (overlaps(S_L, sbytes, q, xb) || overlaps(S_L, sbytes, k, xb) || overlaps(S_L, sbytes, v, xb) ||
+                overlaps(S_L, sbytes, beta, bb) || overlaps(S_L, sbytes, o, ob) ||
+                (S0 && S0 != S_L && overlaps(S_L, sbytes, S0, sbytes))))
+        return EFLA_ERR_ALIAS;
+    void *scratch = noalloc_scratch_ptr();
+    if (!scratch) return EFLA_ERR_CUDA;
+    const bool eu = mode == EFLA_MODE_EULER;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    EFLA_DISPATCH(launch_chunk_simt, dtype, o_dtype, d_k, q, k, v, beta, S0, o, S_L, bh, L, scratch, eu, st);
+}
+
+}  // extern "C"

@@ -156,6 +156,42 @@ efla_status_t efla_decode_step(const void *q, const void *k, const void *v,
                                efla_dtype_t o_dtype, int B, int H, int d_k,
                                int d_v, efla_stream_t stream);
 
+/*
+ * efla_chunk_fwd_noalloc - the same prefill as efla_chunk_fwd, for callers
+ * that cannot allocate device memory.  The pages describe no such call; it
+ * exists for this library's users.  Some hosts (inference engines and
+ * plugins that budget every byte of GPU memory through their own pool, or
+ * latency-critical loops where cudaMalloc/cudaFree would synchronise the
+ * device) cannot hand this library a scratch buffer or let it allocate one.
+ * This entry point takes no workspace and allocates nothing: its scratch is
+ * a fixed array of EFLA_NOALLOC_SCRATCH_BYTES (32 MiB) that the library
+ * places in device memory of every GPU on which it is loaded and keeps until
+ * the process exits.
+ *   Arguments, layouts and results are those of efla_chunk_fwd.  It always
+ *   runs the CUDA-core (exact fp32) chunked kernels, for every dtype and head
+ *   size.  Problems whose scratch would not fit
+ *   (efla_chunk_fwd_workspace_size_simt > EFLA_NOALLOC_SCRATCH_BYTES, e.g.
+ *   more than 409 head-chunks of 64 tokens at d = 128) return
+ *   EFLA_ERR_WORKSPACE before anything is launched.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before capturing a stream
+ *   into a CUDA graph.
+ *   Every call on a device shares the one array and leaves its contents
+ *   behind; nothing in it needs to start zeroed.  Calls whose kernels overlap
+ *   on the GPU (other streams, other host threads) race on it: serialise them.
+ */
+#define EFLA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* Scratch bytes the CUDA-core chunked kernels need for these sizes. */
+size_t efla_chunk_fwd_workspace_size_simt(int B, int H, int L, int d_k, int d_v);
+
+efla_status_t efla_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                     efla_dtype_t dtype, efla_mode_t mode,
+                                     const float *beta, const float *S0,
+                                     void *o, efla_dtype_t o_dtype, float *S_L,
+                                     int B, int H, int L, int d_k, int d_v,
+                                     efla_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
