@@ -63,7 +63,7 @@ constexpr uint32_t OFF_SB = OFF_TLO + SLOT;     // S tile bf16 hi, then lo (MN-m
 constexpr uint32_t OFF_DB = OFF_SB + 4 * SLOT;  // D bf16 hi, then lo (MN-major B), 64 x 64 each
 constexpr uint32_t OFF_ALPHA = OFF_DB + 2 * SLOT;
 constexpr uint32_t OFF_BAR = OFF_ALPHA + 256;
-constexpr uint32_t NBAR = 16;
+constexpr uint32_t NBAR = 18;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -87,12 +87,37 @@ enum : int {
     B_DELTA = 12,   // bf16 D written
     B_SFULL = 13,   // S += K^T D and O += M D done
     B_DRAIN = 14,   // final drain of the MMA pipe
+    B_OREAD = 15,   // [2] state has read O of a chunk out of Y buffer b (one
+                    // completion per two chunks, so a parity test never sees
+                    // it two phases ahead of the issuer)
 };
 
 constexpr uint32_t ID_G = ptx::idesc_bf16(128, 64, false, false);
 constexpr uint32_t ID_YW = ptx::idesc_bf16(128, 128, false, true);
 constexpr uint32_t ID_N64 = ptx::idesc_bf16(128, 64, false, true);
 constexpr uint32_t ID_S = ptx::idesc_bf16(128, 64, true, true);
+
+// Optional timeline trace (compile with -DEFLA_TRACE): the leader thread of
+// each role in CTA 0 stamps clock64() at its hand-off points into
+// g_efla_trace[]: entry = event << 56 | chunk << 40 | (clock & 2^40-1).
+#ifdef EFLA_TRACE
+__device__ unsigned long long g_efla_trace[1 << 16];
+__device__ unsigned int g_efla_trace_n;
+#define EFLA_TR(ev, chunk)                                                                              \
+    do {                                                                                              \
+        if (blockIdx.x == 0) {                                                                        \
+            const unsigned i_ = atomicAdd(&g_efla_trace_n, 1u);                                       \
+            if (i_ < (1u << 16))                                                                      \
+                g_efla_trace[i_] = ((unsigned long long)(ev) << 56) |                                 \
+                                   ((unsigned long long)(chunk) << 40) |                              \
+                                   ((unsigned long long)clock64() & ((1ull << 40) - 1));              \
+        }                                                                                             \
+    } while (0)
+#else
+#define EFLA_TR(ev, chunk) \
+    do {                   \
+    } while (0)
+#endif
 
 __device__ __forceinline__ bool bar_any(uint32_t id, uint32_t n, bool v) {
     uint32_t r;
@@ -117,16 +142,26 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
     }
 }
 
-// Row r of a 64 x 64 fp32 matrix stored as two 32-row halves.
+// A 64 x 64 fp32 matrix stored as two 32-row halves of 256-byte rows.  The
+// 16-byte slots of row r are XOR-permuted by (r & 15), so row-per-thread
+// float4 stores and same-column loads across rows hit distinct banks.
 struct Split64 {
     float *lo, *hi;
     __device__ __forceinline__ float *row(int r) const { return (r < 32 ? lo : hi) + (r & 31) * LDF; }
+    // element (r, c); for c % 4 == 0 this is the start of a contiguous float4
+    __device__ __forceinline__ float *at(int r, int c) const {
+        return row(r) + ((((c >> 2) ^ (r & 15)) << 2) | (c & 3));
+    }
 };
 
-// T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A, by 16 x 16
-// diagonal blocks (right-looking forward substitution, one warp per block)
-// followed by three block rows  T_I,<I = -T_II (A_I,<I T_<I,<I).  Row block I
-// of A is overwritten by the intermediate product.  128 threads (prep).
+// T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A.  First the
+// four 16 x 16 diagonal blocks by right-looking forward substitution (one
+// warp per block, one column per lane pair); then block rows I = 1..3:
+//     R = A_{I,<I} T_{<I,<I},   T_{I,<I} = -T_II R.
+// In the block-row products thread p owns row p/8 of the block row and the
+// 8 consecutive columns 8 (p%8) .. +7, so every step is one scalar and two
+// float4 loads feeding 8 independent FMA chains.  R is parked in row block
+// I of A, which nothing reads afterwards.  128 threads (prep).
 __device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af, const Split64 Tf) {
     {
         const int w = p >> 5, l = p & 31, c = l & 15, h = l >> 4, base = 16 * w;
@@ -137,50 +172,55 @@ __device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af,
         for (int m = 0; m < 16; ++m) {
             const float x = __shfl_sync(0xffffffffu, acc[m >> 1], ((m & 1) << 4) | c);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) acc[s] = fmaf(-Af.row(base + 2 * s + h)[base + m], x, acc[s]);
+            for (int s = 0; s < 8; ++s) acc[s] = fmaf(-*Af.at(base + 2 * s + h, base + m), x, acc[s]);
         }
 #pragma unroll
-        for (int s = 0; s < 8; ++s) Tf.row(base + 2 * s + h)[base + c] = acc[s];
+        for (int s = 0; s < 8; ++s) *Tf.at(base + 2 * s + h, base + c) = acc[s];
     }
     ptx::named_bar(1, 128);
+    const int i = p >> 3, j0 = 8 * (p & 7);
 #pragma unroll 1
     for (int I = 1; I < 4; ++I) {
-        const int W = 16 * I, nent = 16 * W;
-        float R[6];
-#pragma unroll
-        for (int k = 0; k < 6; ++k) {
-            const int e = p + 128 * k;
-            float acc = 0.f;
-            if (e < nent) {
-                const int i = e / W, j = e % W;
-                const float *arow = Af.row(16 * I + i);
-                for (int m = (j & ~15); m < W; ++m) acc = fmaf(arow[m], Tf.row(m)[j], acc);
+        const int W = 16 * I;
+        const bool active = j0 < W;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (active) {
+#pragma unroll 4
+            for (int m = j0 & ~15; m < W; ++m) {
+                const float a = *Af.at(16 * I + i, m);
+                const float4 t0 = *reinterpret_cast<const float4 *>(Tf.at(m, j0));
+                const float4 t1 = *reinterpret_cast<const float4 *>(Tf.at(m, j0 + 4));
+                acc[0] = fmaf(a, t0.x, acc[0]); acc[1] = fmaf(a, t0.y, acc[1]);
+                acc[2] = fmaf(a, t0.z, acc[2]); acc[3] = fmaf(a, t0.w, acc[3]);
+                acc[4] = fmaf(a, t1.x, acc[4]); acc[5] = fmaf(a, t1.y, acc[5]);
+                acc[6] = fmaf(a, t1.z, acc[6]); acc[7] = fmaf(a, t1.w, acc[7]);
             }
-            R[k] = acc;
         }
         ptx::named_bar(1, 128);
-#pragma unroll
-        for (int k = 0; k < 6; ++k) {
-            const int e = p + 128 * k;
-            if (e < nent) Af.row(16 * I + e / W)[e % W] = R[k];
+        if (active) {
+            *reinterpret_cast<float4 *>(Af.at(16 * I + i, j0)) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            *reinterpret_cast<float4 *>(Af.at(16 * I + i, j0 + 4)) = make_float4(acc[4], acc[5], acc[6], acc[7]);
         }
         ptx::named_bar(1, 128);
+        if (active) {
 #pragma unroll
-        for (int k = 0; k < 6; ++k) {
-            const int e = p + 128 * k;
-            if (e < nent) {
-                const int i = e / W, j = e % W;
-                const float *trow = Tf.row(16 * I + i) + 16 * I;
-                float acc = 0.f;
-                for (int m = 0; m <= i; ++m) acc = fmaf(trow[m], Af.row(16 * I + m)[j], acc);
-                Tf.row(16 * I + i)[j] = -acc;
+            for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+            for (int m = 0; m <= i; ++m) {
+                const float t = *Tf.at(16 * I + i, 16 * I + m);
+                const float4 r0 = *reinterpret_cast<const float4 *>(Af.at(16 * I + m, j0));
+                const float4 r1 = *reinterpret_cast<const float4 *>(Af.at(16 * I + m, j0 + 4));
+                acc[0] = fmaf(t, r0.x, acc[0]); acc[1] = fmaf(t, r0.y, acc[1]);
+                acc[2] = fmaf(t, r0.z, acc[2]); acc[3] = fmaf(t, r0.w, acc[3]);
+                acc[4] = fmaf(t, r1.x, acc[4]); acc[5] = fmaf(t, r1.y, acc[5]);
+                acc[6] = fmaf(t, r1.z, acc[6]); acc[7] = fmaf(t, r1.w, acc[7]);
             }
+            *reinterpret_cast<float4 *>(Tf.at(16 * I + i, j0)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+            *reinterpret_cast<float4 *>(Tf.at(16 * I + i, j0 + 4)) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
         }
         ptx::named_bar(1, 128);
     }
 }
 
-// bf16 hi + lo split of a pair of fp32 values (hi = rn(x), lo = rn(x - hi)).
 // One 64-value fp32 row (held as two 32-register halves) -> bf16 hi at
 // `base` and lo at `base + lo_off`, row `row` of a 128-byte-swizzled tile.
 __device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo_off, int row, const uint32_t (&a)[32],
@@ -247,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar[B_DELTA], 128);
         mbar_init(&bar[B_SFULL], 1);
         mbar_init(&bar[B_DRAIN], 1);
+        mbar_init(&bar[B_OREAD], 128);
+        mbar_init(&bar[B_OREAD + 1], 128);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -268,31 +310,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ prep
         const int p = threadIdx.x;
         const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+        float beta_next = ((p & 1) == 0 && (p >> 1) < L) ? __ldg(beta + bh * (long)L + (p >> 1)) : 0.f;
         for (int n = 0; n < nc; ++n) {
             const int s = n & 1;
             unsigned char *st = sm + s * STAGE;
             const int t0 = n * C;
             bool ok = mbar_wait(&bar[B_FULL + s], (n >> 1) & 1, abort_flag);
+            if (p == 0) EFLA_TR(1, n);
             if (bar_any(1, 128, !ok || *abort_flag)) break;
             {   // gate: two lanes per key row, each over one 64-wide half
                 const int r = p >> 1, h = p & 1;
                 const unsigned char *krow = st + (h ? BOXSTRIDE : 0) + SL_K0 * SLOT + r * 128;
                 float ss = 0.f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 8; ++j) {  // visit the row's chunks in swizzled order: no bank conflicts
                     float f[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(krow + 16 * j), f);
+                    unpack8(*reinterpret_cast<const uint4 *>(krow + 16 * (j ^ (r & 7))), f);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
                 }
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                if (h == 0) {
-                    const int t = t0 + r;
-                    alpha_s[r] = (t < L) ? gate_alpha(beta[bh * (long)L + t], ss, euler != 0) : 0.f;
-                }
+                if (h == 0) alpha_s[r] = (t0 + r < L) ? gate_alpha(beta_next, ss, euler != 0) : 0.f;
+                // prefetch next chunk's beta so its global latency is off the critical path
+                const int tn = t0 + C + r;
+                beta_next = (h == 0 && tn < L) ? __ldg(beta + bh * (long)L + tn) : 0.f;
             }
             named_bar(1, 128);
             ok = mbar_wait(&bar[B_GFULL], n & 1, abort_flag);
+            if (p == 0) EFLA_TR(2, n);
             if (bar_any(1, 128, !ok || *abort_flag)) break;
             tc_fence_after();
             uint32_t ga[32], gb[32];
@@ -306,7 +351,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                              reinterpret_cast<float *>(st + SL_W0 * SLOT + BOXSTRIDE)};
             if (p < 64) {  // A row p = alpha_p * (K K^T)[p][c] for c < p
                 const float ap = alpha_s[p];
-                float *arow = Af.row(p);
 #pragma unroll
                 for (int c = 0; c < 64; c += 4) {
                     float4 v;
@@ -316,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t bits = (c + e < 32) ? ga[c + e] : gb[c + e - 32];
                         vv[e] = (c + e < p) ? ap * __uint_as_float(bits) : 0.f;
                     }
-                    *reinterpret_cast<float4 *>(arow + c) = v;
+                    *reinterpret_cast<float4 *>(Af.at(p, c)) = v;
                 }
             } else {       // M row r = (Q K^T)[r][c] for c <= r, as bf16 hi and lo boxes
                 const int r = p - 64;
@@ -337,19 +381,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             named_bar(1, 128);
+            if (p == 0) EFLA_TR(3, n);
             invert_unit_lower(p, Af, Tf);
+            if (p == 0) EFLA_TR(4, n);
             // T' = T diag(alpha) as bf16 hi/lo into the boxes T itself occupies:
             // gather this thread's 32 values first, then overwrite.
             uint32_t th[16], tlo[16];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int e = p + 128 * i, r = e >> 3, j = e & 7;
-                const float *trow = Tf.row(r);
+                const float4 ta = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * j));
+                const float4 tb = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * j + 4));
+                const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const int c0 = 8 * j + 2 * u;
-                    const float x0 = (c0 <= r) ? trow[c0] * alpha_s[c0] : 0.f;
-                    const float x1 = (c0 + 1 <= r) ? trow[c0 + 1] * alpha_s[c0 + 1] : 0.f;
+                    const float x0 = (c0 <= r) ? tv[2 * u] * alpha_s[c0] : 0.f;
+                    const float x1 = (c0 + 1 <= r) ? tv[2 * u + 1] * alpha_s[c0 + 1] : 0.f;
                     split2(x0, x1, th[4 * i + u], tlo[4 * i + u]);
                 }
             }
@@ -364,7 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async();
             mbar_arrive(&bar[B_XFULL]);
+            if (p == 0) EFLA_TR(5, n);
             ok = mbar_wait(&bar[B_YFULL], n & 1, abort_flag);
+            if (p == 0) EFLA_TR(6, n);
             if (bar_any(1, 128, !ok || *abort_flag)) break;
             tc_fence_after();
             if (warp >= 2) {  // W rows live in TMEM lanes 64..127: write -W into the stage
@@ -394,6 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bar[B_A2FULL + (n & 1)]);
+            if (p == 64) EFLA_TR(7, n);
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------ state
@@ -423,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int b = n & 1;
             const int t0 = n * C;
             bool ok = mbar_wait(&bar[B_DFULL], n & 1, abort_flag);
+            if (q == 64) EFLA_TR(10, n);
             if (bar_any(2, 128, !ok || *abort_flag)) break;
             tc_fence_after();
             if (warp >= 6) {  // D rows (lanes 64..127) -> bf16 MN-major operand, row c = lane - 64
@@ -437,7 +489,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bar[B_DELTA]);
+            if (q == 64) EFLA_TR(11, n);
             ok = mbar_wait(&bar[B_SFULL], n & 1, abort_flag);
+            if (q == 64) EFLA_TR(12, n);
             if (bar_any(2, 128, !ok || *abort_flag)) break;
             tc_fence_after();
             uint32_t sa[32], sb[32];
@@ -449,6 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bar[B_SBFULL]);
+            if (q == 64) EFLA_TR(13, n);
             if (warp < 6) {  // O rows (lanes 0..63)
                 uint32_t oa[32], ob[32];
                 tmem_ld32(tl + T_YU + 64 * b, oa);
@@ -465,6 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&bar[B_OREAD + (n & 1)]);
+            if (q == 0) EFLA_TR(14, n);
             if (n == nc - 1 && SL) {
                 float *dst = SL + ((size_t)bh * DK + q) * DK + j0;
 #pragma unroll
@@ -539,41 +597,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(&bar[B_SFULL]);
                 mma_commit(&bar[B_EMPTY + (n & 1)]);
             };
-            bool ok = true;
-            do {
-                if (!(ok = mbar_wait(&bar[B_FULL], 0, abort_flag))) break;
-                tc_fence_after();
-                issue_G(0);
-                if (!(ok = mbar_wait(&bar[B_XFULL], 0, abort_flag))) break;
-                tc_fence_after();
-                issue_Y(0);
-                if (nc > 1) {
-                    if (!(ok = mbar_wait(&bar[B_FULL + 1], 0, abort_flag))) break;
-                    if (!(ok = mbar_wait(&bar[B_GEMPTY], 0, abort_flag))) break;
+            // Event-driven issue: each product goes out as soon as its inputs are
+            // ready, the serial D / SO chain first, so Y(n+1) and G(n+2) fill the
+            // gaps while the state warps read TMEM.  Ordering rules:
+            //   D(n)  after -W/M of chunk n (a2) and the bf16 state (sb);
+            //   SO(n) after the bf16 D (delta);
+            //   Y(m)  after X(m) and after O(m-2) left the Y buffer (oread[m%2]);
+            //   G(m)  after its TMA stage landed, G(m-1) was read (gempty) and
+            //         SO(m-2) was issued (so the commit that signals G(m)
+            //         also covers every earlier reader of the buffers that
+            //         chunk m's prep overwrites).
+            int nD = 0, nS = 0, nY = 0, nG = 0;
+            long long idle_since = clock64();
+            while (nS < nc) {
+                bool did = false;
+                if (nD < nc && nD == nS && nD < nY && mbar_test(&bar[B_A2FULL + (nD & 1)], (nD >> 1) & 1) &&
+                    mbar_test(&bar[B_SBFULL], nD & 1)) {
                     tc_fence_after();
-                    issue_G(1);
+                    EFLA_TR(20, nD); issue_D(nD++);
+                    did = true;
                 }
-                for (int n = 0; n < nc; ++n) {
-                    if (!(ok = mbar_wait(&bar[B_A2FULL + (n & 1)], (n >> 1) & 1, abort_flag))) break;
-                    if (!(ok = mbar_wait(&bar[B_SBFULL], n & 1, abort_flag))) break;
+                if (nS < nD && mbar_test(&bar[B_DELTA], nS & 1)) {
                     tc_fence_after();
-                    issue_D(n);
-                    if (!(ok = mbar_wait(&bar[B_DELTA], n & 1, abort_flag))) break;
-                    tc_fence_after();
-                    issue_SO(n);
-                    if (n + 1 < nc) {
-                        if (!(ok = mbar_wait(&bar[B_XFULL], (n + 1) & 1, abort_flag))) break;
-                        tc_fence_after();
-                        issue_Y(n + 1);
-                    }
-                    if (n + 2 < nc) {
-                        if (!(ok = mbar_wait(&bar[B_FULL + (n & 1)], ((n + 2) >> 1) & 1, abort_flag))) break;
-                        if (!(ok = mbar_wait(&bar[B_GEMPTY], (n + 1) & 1, abort_flag))) break;
-                        tc_fence_after();
-                        issue_G(n + 2);
-                    }
+                    EFLA_TR(21, nS); issue_SO(nS++);
+                    did = true;
                 }
-            } while (0);
+                if (nY < nc && nY < nG && nY <= nD + 1 && mbar_test(&bar[B_XFULL], nY & 1) &&
+                    (nY < 2 || mbar_test(&bar[B_OREAD + (nY & 1)], ((nY - 2) >> 1) & 1))) {
+                    tc_fence_after();
+                    EFLA_TR(22, nY); issue_Y(nY++);
+                    did = true;
+                }
+                if (nG < nc && nG <= nS + 1 && nG <= nY + 1 && mbar_test(&bar[B_FULL + (nG & 1)], (nG >> 1) & 1) &&
+                    (nG == 0 || mbar_test(&bar[B_GEMPTY], (nG - 1) & 1))) {
+                    tc_fence_after();
+                    EFLA_TR(23, nG); issue_G(nG++);
+                    did = true;
+                }
+                if (did) {
+                    idle_since = clock64();
+                } else if (*abort_flag) {
+                    break;
+                } else if (clock64() - idle_since > kWaitCycles) {
+                    *abort_flag = 1;
+                    raise_error(kErrTimeout);
+                    break;
+                }
+            }
             // drain: wait (bounded, even after an abort) until every MMA issued has completed
             mma_commit(&bar[B_DRAIN]);
             int never = 0;

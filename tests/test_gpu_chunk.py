@@ -24,6 +24,7 @@ def run(efla, x, mode="exact", S0=None, out_dtype=torch.float32):
     o, SL = efla.chunk_fwd(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), x["beta"].cuda(),
                            None if S0 is None else S0.cuda(), mode=mode, out_dtype=out_dtype)
     torch.cuda.synchronize()
+    assert efla.last_error() == 0, "a device-side wait timed out"
     return o, SL
 
 

@@ -24,6 +24,7 @@ def check_heads(efla, x, dtype, heads=None):
     S0 = None if x["S0"] is None else x["S0"].cuda()
     o, SL = efla.chunk_fwd(q, k, v, beta, S0)
     torch.cuda.synchronize()
+    assert efla.last_error() == 0, "a device-side wait timed out"
     B, H = x["q"].shape[:2]
     pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
     for b, h in pairs:
