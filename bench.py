@@ -167,13 +167,25 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Max of a per-rank scalar over all ranks (the slowest rank's time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(w, rank: int) -> int:
+    """Each rank draws its own independent (b,h) problems."""
+    return 42 + w.index + 1000 * rank
+
+
+def job_tokens_per_s(world: int, B: int, L: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processed B*L tokens per step; time is
+    the slowest rank's."""
+    return world * B * L * steps / (ms_max / 1e3)
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -243,7 +255,7 @@ def run_ours(args):
     peaks = load_peaks()
     w = workloads.WORKLOADS[WORKLOAD]
     B, H, L, d = w.B, w.H, w.L, w.d
-    x = workloads.chunk_inputs(w, seed=42 + w.index + 1000 * rank)
+    x = workloads.chunk_inputs(w, seed=rank_seed(w, rank))
     sets = []
     for _ in range(ROTATE):
         s = {n: x[n].to(dev) for n in ("q", "k", "v", "beta")}
@@ -288,7 +300,7 @@ def run_ours(args):
     ms = e0.elapsed_time(e1)
     ms_max = max_over_ranks(ms, world)
     ms_step = ms_max / args.steps
-    value = world * B * L * args.steps / (ms_max / 1e3)
+    value = job_tokens_per_s(world, B, L, args.steps, ms_max)
     del graphs
 
     # roofline of the dominant kernel (the whole efla_chunk_fwd when it is one launch)

@@ -41,7 +41,7 @@ STATUS = {0: "EFLA_OK", 1: "EFLA_ERR_NULL", 2: "EFLA_ERR_SHAPE", 3: "EFLA_ERR_DT
           9: "EFLA_ERR_ALIAS"}
 EXPORTS = ("efla_status_string", "efla_version", "efla_last_error", "efla_gate",
            "efla_chunk_fwd_workspace_size", "efla_chunk_fwd", "efla_decode_step",
-           "efla_chunk_fwd_workspace_size_simt", "efla_chunk_fwd_noalloc")
+           "efla_chunk_fwd_workspace_size_simt", "efla_chunk_fwd_noalloc", "efla_diag_wait_timeout")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _p, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -61,6 +61,8 @@ _lib.efla_chunk_fwd_workspace_size_simt.restype = _sz
 _lib.efla_chunk_fwd_workspace_size_simt.argtypes = [_i, _i, _i, _i, _i]
 _lib.efla_chunk_fwd_noalloc.restype = _i
 _lib.efla_chunk_fwd_noalloc.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _p]
+_lib.efla_diag_wait_timeout.restype = _i
+_lib.efla_diag_wait_timeout.argtypes = [ctypes.c_longlong, _p]
 _lib.efla_decode_step.restype = _i
 _lib.efla_decode_step.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 

@@ -123,9 +123,29 @@ size_t simt_workspace_bytes(long bh, int L, int d) {
         return F<__nv_bfloat16, __nv_bfloat16, 128>(__VA_ARGS__);                                 \
     } while (0)
 
+// One mbarrier that nobody arrives on, waited on with the prefill kernel's
+// bounded wait: exercises the timeout path end to end.
+__global__ void diag_wait_timeout_kernel(long long limit_cycles) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        efla::ptx::mbar_init(&bar, 1);
+        efla::ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) efla::ptx::mbar_wait(&bar, 0, &abort_flag, limit_cycles);
+}
+
 }  // namespace
 
 extern "C" {
+
+efla_status_t efla_diag_wait_timeout(long long limit_cycles, efla_stream_t stream) {
+    if (limit_cycles <= 0 || limit_cycles > 8000000000LL) return EFLA_ERR_SHAPE;
+    diag_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
+    return launched();
+}
 
 const char *efla_status_string(efla_status_t s) {
     switch (s) {

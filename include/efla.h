@@ -90,6 +90,16 @@ int efla_version(void);
 efla_status_t efla_last_error(void);
 
 /*
+ * Diagnostic: launch one CTA that waits on an mbarrier nothing ever arrives
+ * on, through the same clock-bounded wait the prefill kernel uses, with a
+ * limit of `limit_cycles` SM clock cycles.  The wait gives up, the kernel
+ * sets the sticky error word and returns; the next efla_last_error()
+ * reports EFLA_ERR_TIMEOUT and the CUDA context stays usable.  Exists so the
+ * failure path can be tested without faulting or hanging a GPU.
+ */
+efla_status_t efla_diag_wait_timeout(long long limit_cycles, efla_stream_t stream);
+
+/*
  * efla_gate - the exact-flow gate (关键设计 2; numerics per 损失函数 /
  * 训练策略): for every row t of k,
  *     lambda[t] = sum_i k[t][i]^2                (fp32 accumulation, unclamped)
