@@ -212,7 +212,7 @@ efla_status_t efla_gate(const void *k, efla_dtype_t dtype, efla_mode_t mode, con
 size_t efla_chunk_fwd_workspace_size(efla_dtype_t dtype, int B, int H, int L, int d_k, int d_v) {
     if (check_common(dtype, EFLA_MODE_EXACT) != EFLA_OK || B <= 0 || H <= 0 || L <= 0) return 0;
     if (check_head(d_k, d_v) != EFLA_OK) return 0;
-    if (tc_path_applies(dtype == EFLA_BF16, d_k, d_v)) return 0;
+    if (tc_path_applies(dtype == EFLA_BF16, d_k, d_v)) return tc::workspace_bytes((long)B * H, L);
     return simt_workspace_bytes((long)B * H, L, d_k);
 }
 
@@ -256,15 +256,14 @@ efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v, efla_d
     const bool eu = mode == EFLA_MODE_EULER;
     const bool bf = dtype == EFLA_BF16;
 
-    if (tc_path_applies(bf, d_k, d_v))
-        return launch_chunk_tc(q, k, v, beta, S0, o, o_dtype == EFLA_BF16, S_L, bh, L, eu, st);
-
-    const size_t need = simt_workspace_bytes(bh, L, d_k);
+    const bool tcp = tc_path_applies(bf, d_k, d_v);
+    const size_t need = tcp ? tc::workspace_bytes(bh, L) : simt_workspace_bytes(bh, L, d_k);
     if (!workspace || workspace_bytes < need) return EFLA_ERR_WORKSPACE;
     if (overlaps(workspace, need, q, xb) || overlaps(workspace, need, k, xb) || overlaps(workspace, need, v, xb) ||
         overlaps(workspace, need, o, ob) || overlaps(workspace, need, beta, bb) ||
         overlaps(workspace, need, S0, sbytes) || overlaps(workspace, need, S_L, sbytes))
         return EFLA_ERR_ALIAS;
+    if (tcp) return launch_chunk_tc(q, k, v, beta, S0, o, o_dtype == EFLA_BF16, S_L, bh, L, eu, workspace, st);
     EFLA_DISPATCH(launch_chunk_simt, dtype, o_dtype, d_k, q, k, v, beta, S0, o, S_L, bh, L, workspace, eu, st);
 }
 

@@ -6,10 +6,13 @@
 // flowchart) chunk by chunk in the UT form of the chunk-parallel scheme that
 // page cites (整体框架, "WY / UT"), with C = 64:
 //
+//   kernel chunk_T_kernel, one CTA per chunk, all chunks in parallel:
 //   alpha = gate(beta, ||k||^2)                       (fp32, CUDA cores)
+//   A  = strictly-lower(diag(alpha) K K^T)            (mma.sync bf16, fp32 acc.)
+//   T  = (I + A)^{-1}                                 (CUDA cores + mma.sync TF32)
+//   X  = [0; T diag(alpha)]                           (bf16 hi + lo, to scratch)
+//   kernel chunk_tc_kernel, serial over the chunks of one (b, h, d_v half):
 //   G  = [K; Q] K^T                                   (tcgen05, M=128 N=64 K=128)
-//   A  = strictly-lower(diag(alpha) K K^T);  T = (I + A)^{-1}   (fp32, CUDA cores)
-//   X  = [0; T diag(alpha)]                           (bf16 hi + lo operands)
 //   [. ; W] = X K,   [0; U] = X V_tile                (tcgen05, N=128 and N=64)
 //   Y += [Q; -W] S  ->  [Q S; U - W S] = [Q S; D]     (tcgen05, N=64 K=128)
 //   S += K^T D                                        (tcgen05, N=64 K=64)
@@ -25,9 +28,12 @@
 // (x = hi + lo to ~16 significant bits); only -W goes in as a single bf16.
 // Accumulation is fp32 in TMEM and the state is kept in fp32.
 //
+// Everything S-independent and per-chunk that is not a tensor-core product
+// (the gate and T) runs in the first kernel, so the serial kernel only moves
+// T' in and keeps its tensor pipe and state chain busy.
 // One CTA per (b, h, half of d_v): the 128 x 64 fp32 state tile lives in
 // TMEM for the whole sequence.  Warp roles:
-//   warps 0-3  "prep":  gate, T, X and -W for chunk n+1 (S-independent)
+//   warps 0-3  "prep":  X in, M and -W for chunk n+1 (S-independent)
 //   warps 4-7  "state": D -> bf16, S -> bf16 and O -> HBM for chunk n
 //   warp 8     one thread issues every tcgen05.mma and commit
 //   warp 9     one thread issues the TMA loads (2-stage K/Q/V ring)
@@ -61,15 +67,12 @@ constexpr uint32_t OFF_Z1 = OFF_THI + SLOT;     // zero box, then T' lo  ([0; T'
 constexpr uint32_t OFF_TLO = OFF_Z1 + SLOT;
 constexpr uint32_t OFF_SB = OFF_TLO + SLOT;     // S tile bf16 hi, then lo (MN-major B), 128 x 64 each
 constexpr uint32_t OFF_DB = OFF_SB + 4 * SLOT;  // D bf16 hi, then lo (MN-major B), 64 x 64 each
-constexpr uint32_t OFF_ALPHA = OFF_DB + 2 * SLOT;
-constexpr uint32_t OFF_BAR = OFF_ALPHA + 256;
-constexpr uint32_t NBAR = 18;
+constexpr uint32_t OFF_BAR = OFF_DB + 2 * SLOT;
+constexpr uint32_t XBYTES = 2 * SLOT;           // T' hi and lo boxes of one chunk (workspace image)
+constexpr uint32_t NBAR = 18;  // indices 0..17
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-// fp32 scratch of the T computation aliases buffers that are idle meanwhile:
-// A (64 x 64) the two W boxes of the stage being prepared (rows 0-31 / 32-63),
-// T (64 x 64) the T' hi / lo boxes (rows 0-31 / 32-63).
 
 // TMEM columns (fp32, 128 lanes)
 constexpr uint32_t T_S = 0, T_G = 64, T_YW = 128, T_YU = 256, TMEM_COLS = 512;
@@ -87,6 +90,7 @@ enum : int {
     B_DELTA = 12,   // bf16 D written
     B_SFULL = 13,   // S += K^T D and O += M D done
     B_DRAIN = 14,   // final drain of the MMA pipe
+    B_OFULL = 17,   // O += M D done
     B_OREAD = 15,   // [2] state has read O of a chunk out of Y buffer b (one
                     // completion per two chunks, so a parity test never sees
                     // it two phases ahead of the issuer)
@@ -97,27 +101,35 @@ constexpr uint32_t ID_YW = ptx::idesc_bf16(128, 128, false, true);
 constexpr uint32_t ID_N64 = ptx::idesc_bf16(128, 64, false, true);
 constexpr uint32_t ID_S = ptx::idesc_bf16(128, 64, true, true);
 
-// Optional timeline trace (compile with -DEFLA_TRACE): the leader thread of
-// each role in CTA 0 stamps clock64() at its hand-off points into
-// g_efla_trace[]: entry = event << 56 | chunk << 40 | (clock & 2^40-1).
+// Optional timeline trace (compile with -DEFLA_TRACE): threads of CTA 0
+// store clock64() at their hand-off points into fixed slots
+// g_efla_trace[chunk % 1024][event] (plain stores, no atomics, so tracing
+// adds no round trip to the critical path).
 #ifdef EFLA_TRACE
-__device__ unsigned long long g_efla_trace[1 << 16];
-__device__ unsigned int g_efla_trace_n;
-#define EFLA_TR(ev, chunk)                                                                              \
-    do {                                                                                              \
-        if (blockIdx.x == 0) {                                                                        \
-            const unsigned i_ = atomicAdd(&g_efla_trace_n, 1u);                                       \
-            if (i_ < (1u << 16))                                                                      \
-                g_efla_trace[i_] = ((unsigned long long)(ev) << 56) |                                 \
-                                   ((unsigned long long)(chunk) << 40) |                              \
-                                   ((unsigned long long)clock64() & ((1ull << 40) - 1));              \
-        }                                                                                             \
+__device__ long long g_efla_trace[1024 * 64];
+#define EFLA_TR(ev, chunk)                                                                   \
+    do {                                                                                   \
+        if (blockIdx.x == 0) g_efla_trace[((chunk) & 1023) * 64 + ((ev) & 63)] = clock64(); \
     } while (0)
 #else
 #define EFLA_TR(ev, chunk) \
     do {                   \
     } while (0)
 #endif
+
+__device__ __forceinline__ uint32_t f2tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// D(16x8) += A(16x8, row) B(8x8, col), TF32 inputs, fp32 accumulation (warp-wide).
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
 
 __device__ __forceinline__ bool bar_any(uint32_t id, uint32_t n, bool v) {
     uint32_t r;
@@ -156,13 +168,13 @@ struct Split64 {
 
 // T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A.  First the
 // four 16 x 16 diagonal blocks by right-looking forward substitution (one
-// warp per block, one column per lane pair); then block rows I = 1..3:
-//     R = A_{I,<I} T_{<I,<I},   T_{I,<I} = -T_II R.
-// In the block-row products thread p owns row p/8 of the block row and the
-// 8 consecutive columns 8 (p%8) .. +7, so every step is one scalar and two
-// float4 loads feeding 8 independent FMA chains.  R is parked in row block
-// I of A, which nothing reads afterwards.  128 threads (prep).
-__device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af, const Split64 Tf) {
+// warp per block, one column per lane pair, fp32); then block rows I = 1..3:
+//     R = A_{I,<I} T_{<I,<I},   T_{I,<I} = -T_II R,
+// as 16 x 8 tiles on mma.sync (TF32 operands, fp32 accumulation).  TF32
+// here costs nothing measurable: T then feeds bf16 hi/lo operands, and an
+// emulation of the whole kernel gave the same error against the oracle
+// with fp32 or TF32 block products.  128 threads (prep).
+__device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af, const Split64 Tf, int n_trace = 0) {
     {
         const int w = p >> 5, l = p & 31, c = l & 15, h = l >> 4, base = 16 * w;
         float acc[8];
@@ -176,47 +188,55 @@ __device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af,
         }
 #pragma unroll
         for (int s = 0; s < 8; ++s) *Tf.at(base + 2 * s + h, base + c) = acc[s];
+        if (l == 0) EFLA_TR(30 + w, n_trace);
     }
     ptx::named_bar(1, 128);
-    const int i = p >> 3, j0 = 8 * (p & 7);
+    // Block rows on the tensor cores through mma.sync m16n8k8 (TF32 inputs,
+    // fp32 accumulation): warp w owns the 8-column tiles jt = w, w+4, ... of
+    // block row I, so R's tile and the T tile computed from it stay inside
+    // one warp.  R is parked in T's own slots between the two products.
+    const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll 1
     for (int I = 1; I < 4; ++I) {
-        const int W = 16 * I;
-        const bool active = j0 < W;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (active) {
-#pragma unroll 4
-            for (int m = j0 & ~15; m < W; ++m) {
-                const float a = *Af.at(16 * I + i, m);
-                const float4 t0 = *reinterpret_cast<const float4 *>(Tf.at(m, j0));
-                const float4 t1 = *reinterpret_cast<const float4 *>(Tf.at(m, j0 + 4));
-                acc[0] = fmaf(a, t0.x, acc[0]); acc[1] = fmaf(a, t0.y, acc[1]);
-                acc[2] = fmaf(a, t0.z, acc[2]); acc[3] = fmaf(a, t0.w, acc[3]);
-                acc[4] = fmaf(a, t1.x, acc[4]); acc[5] = fmaf(a, t1.y, acc[5]);
-                acc[6] = fmaf(a, t1.z, acc[6]); acc[7] = fmaf(a, t1.w, acc[7]);
+        const int r0 = 16 * I;
+#pragma unroll 1
+        for (int jt = w; jt < 2 * I; jt += 4) {
+            const int c0 = 8 * jt;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            // R tile = A[r0.., k] T[k, c0..] over k from the column's own block up to r0
+#pragma unroll 1
+            for (int k0 = 16 * (jt >> 1); k0 < r0; k0 += 8) {
+                const uint32_t a[4] = {f2tf32(*Af.at(r0 + g, k0 + t)), f2tf32(*Af.at(r0 + g + 8, k0 + t)),
+                                       f2tf32(*Af.at(r0 + g, k0 + t + 4)), f2tf32(*Af.at(r0 + g + 8, k0 + t + 4))};
+                const uint32_t bb[2] = {f2tf32(*Tf.at(k0 + t, c0 + g)), f2tf32(*Tf.at(k0 + t + 4, c0 + g))};
+                mma_tf32(acc, a, bb);
             }
-        }
-        ptx::named_bar(1, 128);
-        if (active) {
-            *reinterpret_cast<float4 *>(Af.at(16 * I + i, j0)) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            *reinterpret_cast<float4 *>(Af.at(16 * I + i, j0 + 4)) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        }
-        ptx::named_bar(1, 128);
-        if (active) {
+            *Tf.at(r0 + g, c0 + 2 * t) = acc[0];
+            *Tf.at(r0 + g, c0 + 2 * t + 1) = acc[1];
+            *Tf.at(r0 + g + 8, c0 + 2 * t) = acc[2];
+            *Tf.at(r0 + g + 8, c0 + 2 * t + 1) = acc[3];
+            __syncwarp();
+            uint32_t rb[2][2];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-            for (int m = 0; m <= i; ++m) {
-                const float t = *Tf.at(16 * I + i, 16 * I + m);
-                const float4 r0 = *reinterpret_cast<const float4 *>(Af.at(16 * I + m, j0));
-                const float4 r1 = *reinterpret_cast<const float4 *>(Af.at(16 * I + m, j0 + 4));
-                acc[0] = fmaf(t, r0.x, acc[0]); acc[1] = fmaf(t, r0.y, acc[1]);
-                acc[2] = fmaf(t, r0.z, acc[2]); acc[3] = fmaf(t, r0.w, acc[3]);
-                acc[4] = fmaf(t, r1.x, acc[4]); acc[5] = fmaf(t, r1.y, acc[5]);
-                acc[6] = fmaf(t, r1.z, acc[6]); acc[7] = fmaf(t, r1.w, acc[7]);
+            for (int kk = 0; kk < 2; ++kk) {
+                rb[kk][0] = f2tf32(*Tf.at(r0 + 8 * kk + t, c0 + g));
+                rb[kk][1] = f2tf32(*Tf.at(r0 + 8 * kk + t + 4, c0 + g));
             }
-            *reinterpret_cast<float4 *>(Tf.at(16 * I + i, j0)) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-            *reinterpret_cast<float4 *>(Tf.at(16 * I + i, j0 + 4)) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
+            __syncwarp();
+            float out[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {  // T tile = -T_II R tile
+                const int k0 = r0 + 8 * kk;
+                const uint32_t a[4] = {f2tf32(*Tf.at(r0 + g, k0 + t)), f2tf32(*Tf.at(r0 + g + 8, k0 + t)),
+                                       f2tf32(*Tf.at(r0 + g, k0 + t + 4)), f2tf32(*Tf.at(r0 + g + 8, k0 + t + 4))};
+                mma_tf32(out, a, rb[kk]);
+            }
+            *Tf.at(r0 + g, c0 + 2 * t) = -out[0];
+            *Tf.at(r0 + g, c0 + 2 * t + 1) = -out[1];
+            *Tf.at(r0 + g + 8, c0 + 2 * t) = -out[2];
+            *Tf.at(r0 + g + 8, c0 + 2 * t + 1) = -out[3];
         }
+        if (lane == 0) EFLA_TR(40 + 4 * I + w, n_trace);
         ptx::named_bar(1, 128);
     }
 }
@@ -226,6 +246,7 @@ __device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af,
 __device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo_off, int row, const uint32_t (&a)[32],
                                                 const uint32_t (&b)[32]);
 
+// bf16 hi + lo split of a pair of fp32 values (hi = rn(x), lo = rn(x - hi)).
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
     const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
     hi = ptx::pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
@@ -252,9 +273,8 @@ __device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo
 template <typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ beta,
-                    const float *__restrict__ S0, Tout *__restrict__ o, float *__restrict__ SL, int L, int nc,
-                    int euler) {
+                    const __grid_constant__ CUtensorMap tm_v, const unsigned char *__restrict__ xws,
+                    const float *__restrict__ S0, Tout *__restrict__ o, float *__restrict__ SL, int L, int nc) {
     using namespace ptx;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
@@ -263,8 +283,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + 4);
-    float *alpha_s = reinterpret_cast<float *>(sm + OFF_ALPHA);
-    const Split64 Tf{reinterpret_cast<float *>(sm + OFF_THI), reinterpret_cast<float *>(sm + OFF_TLO)};
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long bh = blockIdx.x / NSPLIT;
@@ -289,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar[B_DRAIN], 1);
         mbar_init(&bar[B_OREAD], 128);
         mbar_init(&bar[B_OREAD + 1], 128);
+        mbar_init(&bar[B_OFULL], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -308,62 +327,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 4) {
         // ------------------------------------------------------------ prep
+        // T' = T diag(alpha) of every chunk arrives precomputed from
+        // chunk_T_kernel as the hi and lo bf16 boxes, already in the swizzled
+        // image the X operand descriptors read.  This role moves it in
+        // (prefetched one chunk ahead in registers), writes M = lower(Q K^T) as
+        // hi/lo boxes, and -W from X K.
         const int p = threadIdx.x;
         const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
-        float beta_next = ((p & 1) == 0 && (p >> 1) < L) ? __ldg(beta + bh * (long)L + (p >> 1)) : 0.f;
+        const uint4 *xsrc = reinterpret_cast<const uint4 *>(xws + (size_t)bh * nc * XBYTES);
+        uint4 xr[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xr[i] = __ldcs(xsrc + p + 128 * i);
         for (int n = 0; n < nc; ++n) {
             const int s = n & 1;
             unsigned char *st = sm + s * STAGE;
-            const int t0 = n * C;
-            bool ok = mbar_wait(&bar[B_FULL + s], (n >> 1) & 1, abort_flag);
-            if (p == 0) EFLA_TR(1, n);
-            if (bar_any(1, 128, !ok || *abort_flag)) break;
-            {   // gate: two lanes per key row, each over one 64-wide half
-                const int r = p >> 1, h = p & 1;
-                const unsigned char *krow = st + (h ? BOXSTRIDE : 0) + SL_K0 * SLOT + r * 128;
-                float ss = 0.f;
+            // T' of chunk n into the [0; T'] operand boxes; Y(n-1), their last
+            // reader, completed before this thread's previous W readout.
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {  // visit the row's chunks in swizzled order: no bank conflicts
-                    float f[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(krow + 16 * (j ^ (r & 7))), f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-                }
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                if (h == 0) alpha_s[r] = (t0 + r < L) ? gate_alpha(beta_next, ss, euler != 0) : 0.f;
-                // prefetch next chunk's beta so its global latency is off the critical path
-                const int tn = t0 + C + r;
-                beta_next = (h == 0 && tn < L) ? __ldg(beta + bh * (long)L + tn) : 0.f;
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t b = 16u * (uint32_t)(p + 128 * i);  // byte offset in the 16 KB image
+                *reinterpret_cast<uint4 *>(sm + (b < SLOT ? OFF_THI + b : OFF_TLO + (b - SLOT))) = xr[i];
             }
-            named_bar(1, 128);
-            ok = mbar_wait(&bar[B_GFULL], n & 1, abort_flag);
+            fence_proxy_async();
+            mbar_arrive(&bar[B_XFULL]);
+            if (p == 0) EFLA_TR(5, n);
+            if (n + 1 < nc) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) xr[i] = __ldcs(xsrc + (size_t)(n + 1) * (XBYTES / 16) + p + 128 * i);
+            }
+            bool ok = mbar_wait(&bar[B_GFULL], n & 1, abort_flag);
             if (p == 0) EFLA_TR(2, n);
             if (bar_any(1, 128, !ok || *abort_flag)) break;
             tc_fence_after();
-            uint32_t ga[32], gb[32];
-            tmem_ld32(tl + T_G, ga);
-            tmem_ld32(tl + T_G + 32, gb);
-            tmem_ld_wait(ga);
-            tmem_ld_wait(gb);
-            tc_fence_before();
-            mbar_arrive(&bar[B_GEMPTY]);
-            const Split64 Af{reinterpret_cast<float *>(st + SL_W0 * SLOT),
-                             reinterpret_cast<float *>(st + SL_W0 * SLOT + BOXSTRIDE)};
-            if (p < 64) {  // A row p = alpha_p * (K K^T)[p][c] for c < p
-                const float ap = alpha_s[p];
-#pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    float4 v;
-                    float *vv = reinterpret_cast<float *>(&v);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t bits = (c + e < 32) ? ga[c + e] : gb[c + e - 32];
-                        vv[e] = (c + e < p) ? ap * __uint_as_float(bits) : 0.f;
-                    }
-                    *reinterpret_cast<float4 *>(Af.at(p, c)) = v;
-                }
-            } else {       // M row r = (Q K^T)[r][c] for c <= r, as bf16 hi and lo boxes
+            if (warp >= 2) {  // M row r = (Q K^T)[r][c] for c <= r (TMEM lanes 64..127), bf16 hi and lo boxes
                 const int r = p - 64;
+                uint32_t ga[32], gb[32];
+                tmem_ld32(tl + T_G, ga);
+                tmem_ld32(tl + T_G + 32, gb);
+                tmem_ld_wait(ga);
+                tmem_ld_wait(gb);
                 unsigned char *mhi = sm + OFF_M + (n & 1) * 2 * SLOT, *mlo = mhi + SLOT;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -380,39 +382,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4 *>(mlo + sw128_chunk(r, j)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
                 }
             }
-            named_bar(1, 128);
+            tc_fence_before();
+            mbar_arrive(&bar[B_GEMPTY]);
             if (p == 0) EFLA_TR(3, n);
-            invert_unit_lower(p, Af, Tf);
-            if (p == 0) EFLA_TR(4, n);
-            // T' = T diag(alpha) as bf16 hi/lo into the boxes T itself occupies:
-            // gather this thread's 32 values first, then overwrite.
-            uint32_t th[16], tlo[16];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int e = p + 128 * i, r = e >> 3, j = e & 7;
-                const float4 ta = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * j));
-                const float4 tb = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * j + 4));
-                const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c0 = 8 * j + 2 * u;
-                    const float x0 = (c0 <= r) ? tv[2 * u] * alpha_s[c0] : 0.f;
-                    const float x1 = (c0 + 1 <= r) ? tv[2 * u + 1] * alpha_s[c0 + 1] : 0.f;
-                    split2(x0, x1, th[4 * i + u], tlo[4 * i + u]);
-                }
-            }
-            named_bar(1, 128);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int e = p + 128 * i, r = e >> 3, j = e & 7;
-                *reinterpret_cast<uint4 *>(sm + OFF_THI + sw128_chunk(r, j)) =
-                    make_uint4(th[4 * i], th[4 * i + 1], th[4 * i + 2], th[4 * i + 3]);
-                *reinterpret_cast<uint4 *>(sm + OFF_TLO + sw128_chunk(r, j)) =
-                    make_uint4(tlo[4 * i], tlo[4 * i + 1], tlo[4 * i + 2], tlo[4 * i + 3]);
-            }
-            fence_proxy_async();
-            mbar_arrive(&bar[B_XFULL]);
-            if (p == 0) EFLA_TR(5, n);
             ok = mbar_wait(&bar[B_YFULL], n & 1, abort_flag);
             if (p == 0) EFLA_TR(6, n);
             if (bar_any(1, 128, !ok || *abort_flag)) break;
@@ -504,6 +476,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&bar[B_SBFULL]);
             if (q == 64) EFLA_TR(13, n);
+            ok = mbar_wait(&bar[B_OFULL], n & 1, abort_flag);
+            if (bar_any(2, 128, !ok || *abort_flag)) break;
+            tc_fence_after();
             if (warp < 6) {  // O rows (lanes 0..63)
                 uint32_t oa[32], ob[32];
                 tmem_ld32(tl + T_YU + 64 * b, oa);
@@ -586,6 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16(tmem + T_S, sdesc_sw128(sa + SL_K0 * SLOT + kk * 2048, BOXSTRIDE, 1024),
                                  sdesc_sw128(dba + part * SLOT + kk * 2048, SLOT, 1024), ID_S, 1);
+                mma_commit(&bar[B_SFULL]);  // the state chain waits only for S
 #pragma unroll
                 for (int part = 0; part < 3; ++part) {
                     const uint32_t ma = (part == 2) ? mlo : mhi, da = dba + (part == 1 ? SLOT : 0);
@@ -594,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16(yu, sdesc_sw128(ma + kk * 32, 16, 1024), sdesc_sw128(da + kk * 2048, SLOT, 1024),
                                  ID_N64, 1);
                 }
-                mma_commit(&bar[B_SFULL]);
+                mma_commit(&bar[B_OFULL]);
                 mma_commit(&bar[B_EMPTY + (n & 1)]);
             };
             // Event-driven issue: each product goes out as soon as its inputs are
@@ -636,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (did) {
                     idle_since = clock64();
-                } else if (*abort_flag) {
+                } else if (__nanosleep(64), *abort_flag) {  // back off: leave the issue slots to the SIMT warps
                     break;
                 } else if (clock64() - idle_since > kWaitCycles) {
                     *abort_flag = 1;
@@ -686,6 +662,108 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------- T' kernel
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+constexpr int KLD = DK + 8;  // padded bf16 row stride of K: conflict-free mma.sync fragment loads
+struct TPrepSmem {
+    __nv_bfloat16 K[C][KLD];
+    float A[C * LDF];
+    float T[C * LDF];
+    float alpha[C];
+};
+
+// Per chunk (rows past L zero): alpha = gate(beta, ||k||^2); A = strictly-lower
+// (diag(alpha) K K^T) by mma.sync bf16 on the 20 lower 16 x 8 tiles;
+// T = (I + A)^{-1}; writes T' = T diag(alpha) as bf16 hi and lo boxes in the
+// 128-byte-swizzled image chunk_tc_kernel's descriptors read.  One CTA of 128
+// threads per (b, h, chunk); independent chunks, so latency hides across CTAs.
+__global__ void __launch_bounds__(128) chunk_T_kernel(const __nv_bfloat16 *__restrict__ k,
+                                                      const float *__restrict__ beta,
+                                                      unsigned char *__restrict__ xws, int L, int nc, int euler) {
+    extern __shared__ __align__(16) unsigned char tsm_raw[];
+    TPrepSmem &sm = *reinterpret_cast<TPrepSmem *>(tsm_raw);
+    const int p = threadIdx.x, w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
+    const long gidx = blockIdx.x;
+    const int chunk = (int)(gidx % nc);
+    const long bh = gidx / nc;
+    const int t0 = chunk * C, n = min(C, L - t0);
+    const __nv_bfloat16 *kc = k + ((size_t)bh * L + t0) * DK;
+    for (int e = p; e < C * (DK / 8); e += 128) {
+        const int r = e / (DK / 8), c8 = (e % (DK / 8)) * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < n) v = __ldg(reinterpret_cast<const uint4 *>(kc + (size_t)r * DK + c8));
+        *reinterpret_cast<uint4 *>(&sm.K[r][c8]) = v;
+    }
+    __syncthreads();
+    {   // gate: two lanes per key row
+        const int r = p >> 1, h = p & 1;
+        float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float f[8];
+            unpack8(*reinterpret_cast<const uint4 *>(&sm.K[r][64 * h + 8 * j]), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc8[e] = fmaf(f[e], f[e], acc8[e]);
+        }
+        float ss = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if (h == 0) sm.alpha[r] = (r < n) ? gate_alpha(beta[bh * (long)L + t0 + r], ss, euler != 0) : 0.f;
+    }
+    __syncthreads();
+    const Split64 Af{sm.A, sm.A + 32 * LDF}, Tf{sm.T, sm.T + 32 * LDF};
+    // the 20 tiles (row tile i of 16, column tile j of 8) on or below the diagonal blocks
+    for (int tile = w; tile < 20; tile += 4) {
+        int i = 0, j = tile;
+        while (j >= 2 * i + 2) {
+            j -= 2 * i + 2;
+            ++i;
+        }
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k0 = 0; k0 < DK; k0 += 16) {
+            const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(&sm.K[16 * i + g][k0 + 2 * t]),
+                                   *reinterpret_cast<const uint32_t *>(&sm.K[16 * i + g + 8][k0 + 2 * t]),
+                                   *reinterpret_cast<const uint32_t *>(&sm.K[16 * i + g][k0 + 2 * t + 8]),
+                                   *reinterpret_cast<const uint32_t *>(&sm.K[16 * i + g + 8][k0 + 2 * t + 8])};
+            const uint32_t b[2] = {*reinterpret_cast<const uint32_t *>(&sm.K[8 * j + g][k0 + 2 * t]),
+                                   *reinterpret_cast<const uint32_t *>(&sm.K[8 * j + g][k0 + 2 * t + 8])};
+            mma_bf16_16816(acc, a, b);
+        }
+        const int r0 = 16 * i + g, r1 = r0 + 8, c0 = 8 * j + 2 * t;
+        *Af.at(r0, c0) = (c0 < r0) ? sm.alpha[r0] * acc[0] : 0.f;
+        *Af.at(r0, c0 + 1) = (c0 + 1 < r0) ? sm.alpha[r0] * acc[1] : 0.f;
+        *Af.at(r1, c0) = (c0 < r1) ? sm.alpha[r1] * acc[2] : 0.f;
+        *Af.at(r1, c0 + 1) = (c0 + 1 < r1) ? sm.alpha[r1] * acc[3] : 0.f;
+    }
+    __syncthreads();
+    invert_unit_lower(p, Af, Tf);
+    unsigned char *dst = xws + (size_t)gidx * XBYTES;
+#pragma unroll
+    for (int ii = 0; ii < 4; ++ii) {
+        const int e = p + 128 * ii, r = e >> 3, jj = e & 7;
+        const float4 ta = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * jj));
+        const float4 tb = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * jj + 4));
+        const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
+        uint32_t h4[4], l4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = 8 * jj + 2 * u;
+            const float x0 = (c <= r) ? tv[2 * u] * sm.alpha[c] : 0.f;
+            const float x1 = (c + 1 <= r) ? tv[2 * u + 1] * sm.alpha[c + 1] : 0.f;
+            split2(x0, x1, h4[u], l4[u]);
+        }
+        *reinterpret_cast<uint4 *>(dst + ptx::sw128_chunk(r, jj)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+        *reinterpret_cast<uint4 *>(dst + SLOT + ptx::sw128_chunk(r, jj)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -718,17 +796,25 @@ inline bool make_map(CUtensorMap *m, const void *base, long bh, int L) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Scratch of the tensor-core path: one T' image (hi + lo boxes) per chunk.
+inline size_t workspace_bytes(long bh, int L) { return (size_t)bh * ((L + C - 1) / C) * XBYTES; }
+
 template <typename Tout>
 inline efla_status_t launch(const void *q, const void *k, const void *v, const float *beta, const float *S0,
-                            void *o, float *SL, long bh, int L, bool euler, cudaStream_t st) {
+                            void *o, float *SL, long bh, int L, bool euler, void *ws, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, bh, L) || !make_map(&mk, k, bh, L) || !make_map(&mv, v, bh, L)) return EFLA_ERR_CUDA;
-    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES)) return EFLA_ERR_CUDA;
+    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES) || !ensure_smem<chunk_T_kernel>(sizeof(TPrepSmem)))
+        return EFLA_ERR_CUDA;
     const long grid = bh * NSPLIT;
-    if (grid > 0x7fffffffL) return EFLA_ERR_SHAPE;
     const int nc = (L + C - 1) / C;
-    chunk_tc_kernel<Tout><<<(unsigned)grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mv, beta, S0, static_cast<Tout *>(o),
-                                                                         SL, L, nc, euler ? 1 : 0);
+    if (grid > 0x7fffffffL || bh * nc > 0x7fffffffL) return EFLA_ERR_SHAPE;
+    unsigned char *xws = static_cast<unsigned char *>(ws);
+    chunk_T_kernel<<<(unsigned)(bh * nc), 128, sizeof(TPrepSmem), st>>>(static_cast<const __nv_bfloat16 *>(k), beta,
+                                                                        xws, L, nc, euler ? 1 : 0);
+    if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
+    chunk_tc_kernel<Tout><<<(unsigned)grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mv, xws, S0, static_cast<Tout *>(o),
+                                                                         SL, L, nc);
     return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
 }
 
@@ -739,9 +825,9 @@ inline bool tc_path_applies(bool bf16, int d_k, int d_v) { return bf16 && d_k ==
 
 inline efla_status_t launch_chunk_tc(const void *q, const void *k, const void *v, const float *beta,
                                      const float *S0, void *o, bool o_bf16, float *SL, long bh, int L, bool euler,
-                                     cudaStream_t st) {
-    return o_bf16 ? tc::launch<__nv_bfloat16>(q, k, v, beta, S0, o, SL, bh, L, euler, st)
-                  : tc::launch<float>(q, k, v, beta, S0, o, SL, bh, L, euler, st);
+                                     void *ws, cudaStream_t st) {
+    return o_bf16 ? tc::launch<__nv_bfloat16>(q, k, v, beta, S0, o, SL, bh, L, euler, ws, st)
+                  : tc::launch<float>(q, k, v, beta, S0, o, SL, bh, L, euler, ws, st);
 }
 
 }  // namespace efla
