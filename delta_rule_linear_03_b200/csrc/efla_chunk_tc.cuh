@@ -33,8 +33,9 @@
 // T' in and keeps its tensor pipe and state chain busy.
 // One CTA per (b, h, half of d_v): the 128 x 64 fp32 state tile lives in
 // TMEM for the whole sequence.  Warp roles:
-//   warps 0-3  "prep":  X in, M and -W for chunk n+1 (S-independent)
-//   warps 4-7  "state": D -> bf16, S -> bf16 and O -> HBM for chunk n
+//   warps 0-1  "io":    T' image in (chunk n+1), O of chunk n-1 out to HBM
+//   warps 2-3  "mw":    M and -W for chunk n+1 (S-independent)
+//   warps 4-7  "state": D -> bf16 and S -> bf16 for chunk n (the serial chain)
 //   warp 8     one thread issues every tcgen05.mma and commit
 //   warp 9     one thread issues the TMA loads (2-stage K/Q/V ring)
 // Every mbarrier wait is bounded; a wait that gives up sets the sticky
@@ -69,7 +70,7 @@ constexpr uint32_t OFF_SB = OFF_TLO + SLOT;     // S tile bf16 hi, then lo (MN-m
 constexpr uint32_t OFF_DB = OFF_SB + 4 * SLOT;  // D bf16 hi, then lo (MN-major B), 64 x 64 each
 constexpr uint32_t OFF_BAR = OFF_DB + 2 * SLOT;
 constexpr uint32_t XBYTES = 2 * SLOT;           // T' hi and lo boxes of one chunk (workspace image)
-constexpr uint32_t NBAR = 18;  // indices 0..17
+constexpr uint32_t NBAR = 19;  // indices 0..18
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -90,7 +91,7 @@ enum : int {
     B_DELTA = 12,   // bf16 D written
     B_SFULL = 13,   // S += K^T D and O += M D done
     B_DRAIN = 14,   // final drain of the MMA pipe
-    B_OFULL = 17,   // O += M D done
+    B_OFULL = 17,   // [2] O += M D done for Y buffer b
     B_OREAD = 15,   // [2] state has read O of a chunk out of Y buffer b (one
                     // completion per two chunks, so a parity test never sees
                     // it two phases ahead of the issuer)
@@ -248,9 +249,12 @@ __device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo
 
 // bf16 hi + lo split of a pair of fp32 values (hi = rn(x), lo = rn(x - hi)).
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-    hi = ptx::pack_bf16(__bfloat162float(h0), __bfloat162float(h1));
-    lo = ptx::pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+    uint32_t h, l;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(x1), "f"(x0));  // x0 -> low half
+    const float h0 = __uint_as_float(h << 16), h1 = __uint_as_float(h & 0xffff0000u);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(l) : "f"(x1 - h1), "f"(x0 - h0));
+    hi = h;
+    lo = l;
 }
 
 __device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo_off, int row, const uint32_t (&a)[32],
@@ -295,19 +299,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar[B_EMPTY], 1);
         mbar_init(&bar[B_EMPTY + 1], 1);
         mbar_init(&bar[B_GFULL], 1);
-        mbar_init(&bar[B_GEMPTY], 128);
-        mbar_init(&bar[B_XFULL], 128);
+        mbar_init(&bar[B_GEMPTY], 64);
+        mbar_init(&bar[B_XFULL], 64);
         mbar_init(&bar[B_YFULL], 1);
-        mbar_init(&bar[B_A2FULL], 128);
-        mbar_init(&bar[B_A2FULL + 1], 128);
+        mbar_init(&bar[B_A2FULL], 64);
+        mbar_init(&bar[B_A2FULL + 1], 64);
         mbar_init(&bar[B_SBFULL], 128);
         mbar_init(&bar[B_DFULL], 1);
         mbar_init(&bar[B_DELTA], 128);
         mbar_init(&bar[B_SFULL], 1);
         mbar_init(&bar[B_DRAIN], 1);
-        mbar_init(&bar[B_OREAD], 128);
-        mbar_init(&bar[B_OREAD + 1], 128);
+        mbar_init(&bar[B_OREAD], 64);
+        mbar_init(&bar[B_OREAD + 1], 64);
         mbar_init(&bar[B_OFULL], 1);
+        mbar_init(&bar[B_OFULL + 1], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -325,47 +330,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp < 4) {
-        // ------------------------------------------------------------ prep
+    if (warp < 2) {
+        // ------------------------------------------------------------ io (warps 0-1)
         // T' = T diag(alpha) of every chunk arrives precomputed from
-        // chunk_T_kernel as the hi and lo bf16 boxes, already in the swizzled
-        // image the X operand descriptors read.  This role moves it in
-        // (prefetched one chunk ahead in registers), writes M = lower(Q K^T) as
-        // hi/lo boxes, and -W from X K.
-        const int p = threadIdx.x;
+        // chunk_T_kernel as hi and lo bf16 boxes, already in the swizzled
+        // image the X operand descriptors read: copy it in (prefetched a
+        // chunk ahead in registers).  Then read O of the previous chunk out
+        // of TMEM lanes 0..63 and store it.
+        const int p = threadIdx.x;  // TMEM lane / chunk row
         const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
         const uint4 *xsrc = reinterpret_cast<const uint4 *>(xws + (size_t)bh * nc * XBYTES);
-        uint4 xr[8];
+        uint4 xr[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xr[i] = __ldcs(xsrc + p + 128 * i);
-        for (int n = 0; n < nc; ++n) {
-            const int s = n & 1;
-            unsigned char *st = sm + s * STAGE;
-            // T' of chunk n into the [0; T'] operand boxes; Y(n-1), their last
-            // reader, completed before this thread's previous W readout.
+        for (int i = 0; i < 16; ++i) xr[i] = __ldcs(xsrc + p + 64 * i);
+        auto read_O = [&](int m) -> bool {
+            const bool ok = mbar_wait(&bar[B_OFULL + (m & 1)], (m >> 1) & 1, abort_flag);
+            if (bar_any(3, 64, !ok || *abort_flag)) return false;
+            tc_fence_after();
+            uint32_t oa[32], ob[32];
+            tmem_ld32(tl + T_YU + 64 * (m & 1), oa);
+            tmem_ld32(tl + T_YU + 64 * (m & 1) + 32, ob);
+            tmem_ld_wait(oa);
+            tmem_ld_wait(ob);
+            tc_fence_before();
+            mbar_arrive(&bar[B_OREAD + (m & 1)]);
+            if (p == 0) EFLA_TR(14, m);
+            if (m * C + p < L) {
+                Tout *dst = o + ((size_t)bh * L + m * C + p) * DK + j0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t b = 16u * (uint32_t)(p + 128 * i);  // byte offset in the 16 KB image
-                *reinterpret_cast<uint4 *>(sm + (b < SLOT ? OFF_THI + b : OFF_TLO + (b - SLOT))) = xr[i];
+                for (int c = 0; c < 64; c += 4) {
+                    const uint32_t *src = (c < 32) ? &oa[c] : &ob[c - 32];
+                    store4(dst + c, make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
+                                                __uint_as_float(src[2]), __uint_as_float(src[3])));
+                }
+            }
+            return true;
+        };
+        bool alive = true;
+        for (int n = 0; n < nc && alive; ++n) {
+            if (n > 0) {  // the [0; T'] boxes are free once Y(n-1) completed
+                const bool ok = mbar_wait(&bar[B_YFULL], (n - 1) & 1, abort_flag);
+                if (bar_any(3, 64, !ok || *abort_flag)) break;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t bo = 16u * (uint32_t)(p + 64 * i);  // byte offset in the 16 KB image
+                *reinterpret_cast<uint4 *>(sm + (bo < SLOT ? OFF_THI + bo : OFF_TLO + (bo - SLOT))) = xr[i];
             }
             fence_proxy_async();
             mbar_arrive(&bar[B_XFULL]);
             if (p == 0) EFLA_TR(5, n);
             if (n + 1 < nc) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) xr[i] = __ldcs(xsrc + (size_t)(n + 1) * (XBYTES / 16) + p + 128 * i);
+                for (int i = 0; i < 16; ++i) xr[i] = __ldcs(xsrc + (size_t)(n + 1) * (XBYTES / 16) + p + 64 * i);
             }
+            if (n > 0) alive = read_O(n - 1);
+        }
+        if (alive && !*abort_flag) read_O(nc - 1);
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ mw (warps 2-3)
+        // M = lower(Q K^T) as hi/lo boxes and -W from X K; both live in TMEM
+        // lanes 64..127, which these warps own.
+        const int r = threadIdx.x - 64;  // chunk row
+        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+        for (int n = 0; n < nc; ++n) {
+            unsigned char *st = sm + (n & 1) * STAGE;
             bool ok = mbar_wait(&bar[B_GFULL], n & 1, abort_flag);
-            if (p == 0) EFLA_TR(2, n);
-            if (bar_any(1, 128, !ok || *abort_flag)) break;
+            if (r == 0) EFLA_TR(2, n);
+            if (bar_any(1, 64, !ok || *abort_flag)) break;
             tc_fence_after();
-            if (warp >= 2) {  // M row r = (Q K^T)[r][c] for c <= r (TMEM lanes 64..127), bf16 hi and lo boxes
-                const int r = p - 64;
+            {
                 uint32_t ga[32], gb[32];
                 tmem_ld32(tl + T_G, ga);
                 tmem_ld32(tl + T_G + 32, gb);
                 tmem_ld_wait(ga);
                 tmem_ld_wait(gb);
+                tc_fence_before();
+                mbar_arrive(&bar[B_GEMPTY]);
                 unsigned char *mhi = sm + OFF_M + (n & 1) * 2 * SLOT, *mlo = mhi + SLOT;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -382,41 +423,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4 *>(mlo + sw128_chunk(r, j)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&bar[B_GEMPTY]);
-            if (p == 0) EFLA_TR(3, n);
+            if (r == 0) EFLA_TR(3, n);
             ok = mbar_wait(&bar[B_YFULL], n & 1, abort_flag);
-            if (p == 0) EFLA_TR(6, n);
-            if (bar_any(1, 128, !ok || *abort_flag)) break;
+            if (r == 0) EFLA_TR(6, n);
+            if (bar_any(1, 64, !ok || *abort_flag)) break;
             tc_fence_after();
-            if (warp >= 2) {  // W rows live in TMEM lanes 64..127: write -W into the stage
-                const int r = p - 64;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t wa[32], wb[32];
-                    tmem_ld32(tl + T_YW + 64 * h, wa);
-                    tmem_ld32(tl + T_YW + 64 * h + 32, wb);
-                    tmem_ld_wait(wa);
-                    tmem_ld_wait(wb);
-                    unsigned char *wrow = st + SL_W0 * SLOT + h * BOXSTRIDE;
+            for (int h = 0; h < 2; ++h) {
+                uint32_t wa[32], wb[32];
+                tmem_ld32(tl + T_YW + 64 * h, wa);
+                tmem_ld32(tl + T_YW + 64 * h + 32, wb);
+                tmem_ld_wait(wa);
+                tmem_ld_wait(wb);
+                unsigned char *wrow = st + SL_W0 * SLOT + h * BOXSTRIDE;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        uint32_t w4[4];
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t w4[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int c0 = 8 * j + 2 * u;
-                            const float x0 = __uint_as_float(c0 < 32 ? wa[c0] : wb[c0 - 32]);
-                            const float x1 = __uint_as_float(c0 + 1 < 32 ? wa[c0 + 1] : wb[c0 + 1 - 32]);
-                            w4[u] = pack_bf16(-x0, -x1);
-                        }
-                        *reinterpret_cast<uint4 *>(wrow + sw128_chunk(r, j)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int c0 = 8 * j + 2 * u;
+                        const float x0 = __uint_as_float(c0 < 32 ? wa[c0] : wb[c0 - 32]);
+                        const float x1 = __uint_as_float(c0 + 1 < 32 ? wa[c0 + 1] : wb[c0 + 1 - 32]);
+                        w4[u] = pack_bf16(-x0, -x1);
                     }
+                    *reinterpret_cast<uint4 *>(wrow + sw128_chunk(r, j)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
             }
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bar[B_A2FULL + (n & 1)]);
-            if (p == 64) EFLA_TR(7, n);
+            if (r == 0) EFLA_TR(7, n);
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------ state
@@ -444,7 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int n = 0; n < nc; ++n) {
             const int b = n & 1;
-            const int t0 = n * C;
             bool ok = mbar_wait(&bar[B_DFULL], n & 1, abort_flag);
             if (q == 64) EFLA_TR(10, n);
             if (bar_any(2, 128, !ok || *abort_flag)) break;
@@ -456,9 +491,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(tl + T_YU + 64 * b + 32, db);
                 tmem_ld_wait(da);
                 tmem_ld_wait(db);
+                if (q == 64) EFLA_TR(15, n);
                 write_split_row(sm + OFF_DB, SLOT, c, da, db);
+                if (q == 64) EFLA_TR(16, n);
             }
             fence_proxy_async();
+            if (q == 64) EFLA_TR(17, n);
             tc_fence_before();
             mbar_arrive(&bar[B_DELTA]);
             if (q == 64) EFLA_TR(11, n);
@@ -471,33 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(tl + T_S + 32, sb);
             tmem_ld_wait(sa);
             tmem_ld_wait(sb);
+            if (q == 64) EFLA_TR(24, n);
             write_split_row(sm + OFF_SB, 2 * SLOT, q, sa, sb);
+            if (q == 64) EFLA_TR(25, n);
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bar[B_SBFULL]);
             if (q == 64) EFLA_TR(13, n);
-            ok = mbar_wait(&bar[B_OFULL], n & 1, abort_flag);
-            if (bar_any(2, 128, !ok || *abort_flag)) break;
-            tc_fence_after();
-            if (warp < 6) {  // O rows (lanes 0..63)
-                uint32_t oa[32], ob[32];
-                tmem_ld32(tl + T_YU + 64 * b, oa);
-                tmem_ld32(tl + T_YU + 64 * b + 32, ob);
-                tmem_ld_wait(oa);
-                tmem_ld_wait(ob);
-                if (t0 + q < L) {
-                    Tout *dst = o + ((size_t)bh * L + t0 + q) * DK + j0;
-#pragma unroll
-                    for (int c = 0; c < 64; c += 4) {
-                        const uint32_t *src = (c < 32) ? &oa[c] : &ob[c - 32];
-                        store4(dst + c, make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
-                                                    __uint_as_float(src[2]), __uint_as_float(src[3])));
-                    }
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&bar[B_OREAD + (n & 1)]);
-            if (q == 0) EFLA_TR(14, n);
             if (n == nc - 1 && SL) {
                 float *dst = SL + ((size_t)bh * DK + q) * DK + j0;
 #pragma unroll
@@ -570,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16(yu, sdesc_sw128(ma + kk * 32, 16, 1024), sdesc_sw128(da + kk * 2048, SLOT, 1024),
                                  ID_N64, 1);
                 }
-                mma_commit(&bar[B_OFULL]);
+                mma_commit(&bar[B_OFULL + (n & 1)]);
                 mma_commit(&bar[B_EMPTY + (n & 1)]);
             };
             // Event-driven issue: each product goes out as soon as its inputs are
@@ -578,7 +596,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // gaps while the state warps read TMEM.  Ordering rules:
             //   D(n)  after -W/M of chunk n (a2) and the bf16 state (sb);
             //   SO(n) after the bf16 D (delta);
-            //   Y(m)  after X(m) and after O(m-2) left the Y buffer (oread[m%2]);
+            //   Y(m)  after X(m), after O(m-2) left the Y buffer (oread[m%2]) and
+            //         after D(m-1) was issued: D(m-1) waits for the -W readout
+            //         of chunk m-1, the last reader of the X K accumulator;
             //   G(m)  after its TMA stage landed, G(m-1) was read (gempty) and
             //         SO(m-2) was issued (so the commit that signals G(m)
             //         also covers every earlier reader of the buffers that
@@ -598,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     EFLA_TR(21, nS); issue_SO(nS++);
                     did = true;
                 }
-                if (nY < nc && nY < nG && nY <= nD + 1 && mbar_test(&bar[B_XFULL], nY & 1) &&
+                if (nY < nc && nY < nG && nY <= nD && mbar_test(&bar[B_XFULL], nY & 1) &&
                     (nY < 2 || mbar_test(&bar[B_OREAD + (nY & 1)], ((nY - 2) >> 1) & 1))) {
                     tc_fence_after();
                     EFLA_TR(22, nY); issue_Y(nY++);
@@ -612,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (did) {
                     idle_since = clock64();
-                } else if (__nanosleep(64), *abort_flag) {  // back off: leave the issue slots to the SIMT warps
+                } else if (*abort_flag) {
                     break;
                 } else if (clock64() - idle_since > kWaitCycles) {
                     *abort_flag = 1;
