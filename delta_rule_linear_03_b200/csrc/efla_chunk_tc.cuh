@@ -70,32 +70,35 @@ constexpr uint32_t OFF_SB = OFF_TLO + SLOT;     // S tile bf16 hi, then lo (MN-m
 constexpr uint32_t OFF_DB = OFF_SB + 4 * SLOT;  // D bf16 hi, then lo (MN-major B), 64 x 64 each
 constexpr uint32_t OFF_BAR = OFF_DB + 2 * SLOT;
 constexpr uint32_t XBYTES = 2 * SLOT;           // T' hi and lo boxes of one chunk (workspace image)
-constexpr uint32_t NBAR = 19;  // indices 0..18
+constexpr uint32_t NBAR = 20;  // indices 0..19
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 // TMEM columns (fp32, 128 lanes)
-constexpr uint32_t T_S = 0, T_G = 64, T_YW = 128, T_YU = 256, TMEM_COLS = 512;
+// X K accumulates into two alternating buffers (YW, by chunk parity) so
+// Y(n+1) can run while the -W readout of chunk n is still pending.
+constexpr uint32_t T_S = 0, T_G = 64, T_YW = 128, T_YU = 384, TMEM_COLS = 512;
 
 enum : int {
     B_FULL = 0,     // [2] TMA stage landed
     B_EMPTY = 2,    // [2] stage free again (commit after the last MMA reading it)
     B_GFULL = 4,    // G ready in TMEM
-    B_GEMPTY = 5,   // prep has read G
-    B_XFULL = 6,    // X written
-    B_YFULL = 7,    // X K and X V done
-    B_A2FULL = 8,   // [2] -W and M written for chunk parity b
-    B_SBFULL = 10,  // bf16 S tile written
-    B_DFULL = 11,   // Y += [Q;-W] S done
-    B_DELTA = 12,   // bf16 D written
-    B_SFULL = 13,   // S += K^T D and O += M D done
-    B_DRAIN = 14,   // final drain of the MMA pipe
-    B_OFULL = 17,   // [2] O += M D done for Y buffer b
-    B_OREAD = 15,   // [2] state has read O of a chunk out of Y buffer b (one
-                    // completion per two chunks, so a parity test never sees
-                    // it two phases ahead of the issuer)
+    B_GEMPTY = 5,   // G read out
+    B_XFULL = 6,    // T' image of the next chunk in place
+    B_YFULL = 7,    // [2] X K and X V of a chunk done (per X K buffer)
+    B_A2FULL = 9,   // [2] -W and M written for chunk parity b
+    B_SBFULL = 11,  // bf16 S tile written
+    B_DFULL = 12,   // Y += [Q;-W] S done
+    B_DELTA = 13,   // bf16 D written
+    B_SFULL = 14,   // S += K^T D done
+    B_DRAIN = 15,   // final drain of the MMA pipe
+    B_OREAD = 16,   // [2] O of a chunk read out of Y buffer b
+    B_OFULL = 18,   // [2] O += M D done for Y buffer b
 };
+// Barriers that complete once per chunk but can be waited on a chunk late
+// come in pairs indexed by chunk parity: each then completes once per two
+// chunks, so a parity wait can never see it two phases ahead.
 
 constexpr uint32_t ID_G = ptx::idesc_bf16(128, 64, false, false);
 constexpr uint32_t ID_YW = ptx::idesc_bf16(128, 128, false, true);
@@ -302,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar[B_GEMPTY], 64);
         mbar_init(&bar[B_XFULL], 64);
         mbar_init(&bar[B_YFULL], 1);
+        mbar_init(&bar[B_YFULL + 1], 1);
         mbar_init(&bar[B_A2FULL], 64);
         mbar_init(&bar[B_A2FULL + 1], 64);
         mbar_init(&bar[B_SBFULL], 128);
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool alive = true;
         for (int n = 0; n < nc && alive; ++n) {
             if (n > 0) {  // the [0; T'] boxes are free once Y(n-1) completed
-                const bool ok = mbar_wait(&bar[B_YFULL], (n - 1) & 1, abort_flag);
+                const bool ok = mbar_wait(&bar[B_YFULL + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_flag);
                 if (bar_any(3, 64, !ok || *abort_flag)) break;
             }
 #pragma unroll
@@ -424,15 +428,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (r == 0) EFLA_TR(3, n);
-            ok = mbar_wait(&bar[B_YFULL], n & 1, abort_flag);
+            ok = mbar_wait(&bar[B_YFULL + (n & 1)], (n >> 1) & 1, abort_flag);
             if (r == 0) EFLA_TR(6, n);
             if (bar_any(1, 64, !ok || *abort_flag)) break;
             tc_fence_after();
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t wa[32], wb[32];
-                tmem_ld32(tl + T_YW + 64 * h, wa);
-                tmem_ld32(tl + T_YW + 64 * h + 32, wb);
+                tmem_ld32(tl + T_YW + 128 * (n & 1) + 64 * h, wa);
+                tmem_ld32(tl + T_YW + 128 * (n & 1) + 64 * h + 32, wb);
                 tmem_ld_wait(wa);
                 tmem_ld_wait(wb);
                 unsigned char *wrow = st + SL_W0 * SLOT + h * BOXSTRIDE;
@@ -533,60 +537,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sba = sbase + OFF_SB, dba = sbase + OFF_DB;
             const uint32_t xhi = sbase + OFF_Z0, xlo = sbase + OFF_Z1;  // [0; T' hi], [0; T' lo]
             auto stage_addr = [&](int n) { return sbase + (uint32_t)(n & 1) * STAGE; };
+            // Descriptors: the 14-bit start-address field holds addr >> 4, and
+            // shared addresses stay below 256 KB, so the field never carries:
+            // the descriptor of (addr + off) is desc(addr) + (off >> 4).  Each group
+            // builds its base descriptors once; the unrolled k-steps add
+            // compile-time offsets, keeping the single issuing thread ahead of
+            // the tensor pipe.
+            const uint64_t dX[2] = {sdesc_sw128(xhi, 16, 1024), sdesc_sw128(xlo, 16, 1024)};
+            const uint64_t dSB = sdesc_sw128(sba, SLOT, 1024), dDB = sdesc_sw128(dba, SLOT, 1024);
             auto issue_G = [&](int n) {
-                const uint32_t sa = stage_addr(n);
+                const uint64_t d0 = sdesc_sw128(stage_addr(n) + SL_K0 * SLOT, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t a = sa + SL_K0 * SLOT + (kk >> 2) * BOXSTRIDE + (kk & 3) * 32;
-                    mma_bf16(tmem + T_G, sdesc_sw128(a, 16, 1024), sdesc_sw128(a, 16, 1024), ID_G, kk > 0);
+                    const uint64_t d = d0 + (((kk >> 2) * BOXSTRIDE + (kk & 3) * 32) >> 4);
+                    mma_bf16(tmem + T_G, d, d, ID_G, kk > 0);
                 }
                 mma_commit(&bar[B_GFULL]);
             };
             auto issue_Y = [&](int n) {  // Y = X_hi [K | V] + X_lo [K | V]
                 const uint32_t sa = stage_addr(n), yu = tmem + T_YU + 64 * (n & 1);
+                const uint64_t dK = sdesc_sw128(sa + SL_K0 * SLOT, BOXSTRIDE, 1024);
+                const uint64_t dV = sdesc_sw128(sa + SL_V * SLOT, SLOT, 1024);
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
-                    const uint32_t xa = part ? xlo : xhi;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + T_YW, sdesc_sw128(xa + kk * 32, 16, 1024),
-                                 sdesc_sw128(sa + SL_K0 * SLOT + kk * 2048, BOXSTRIDE, 1024), ID_YW, part | kk);
+                        mma_bf16(tmem + T_YW + 128 * (n & 1), dX[part] + ((kk * 32) >> 4), dK + ((kk * 2048) >> 4),
+                                 ID_YW, part | kk);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(yu, sdesc_sw128(xa + kk * 32, 16, 1024),
-                                 sdesc_sw128(sa + SL_V * SLOT + kk * 2048, SLOT, 1024), ID_N64, part | kk);
+                        mma_bf16(yu, dX[part] + ((kk * 32) >> 4), dV + ((kk * 2048) >> 4), ID_N64, part | kk);
                 }
-                mma_commit(&bar[B_YFULL]);
+                mma_commit(&bar[B_YFULL + (n & 1)]);
             };
             auto issue_D = [&](int n) {  // Y += [Q; -W] (S_hi + S_lo)
-                const uint32_t sa = stage_addr(n), yu = tmem + T_YU + 64 * (n & 1);
+                const uint32_t yu = tmem + T_YU + 64 * (n & 1);
+                const uint64_t dA = sdesc_sw128(stage_addr(n) + SL_Q0 * SLOT, 16, 1024);
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t a = sa + SL_Q0 * SLOT + (kk >> 2) * BOXSTRIDE + (kk & 3) * 32;
-                        mma_bf16(yu, sdesc_sw128(a, 16, 1024),
-                                 sdesc_sw128(sba + part * 2 * SLOT + kk * 2048, SLOT, 1024), ID_N64, 1);
-                    }
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(yu, dA + (((kk >> 2) * BOXSTRIDE + (kk & 3) * 32) >> 4),
+                                 dSB + ((part * 2 * SLOT + kk * 2048) >> 4), ID_N64, 1);
                 mma_commit(&bar[B_DFULL]);
             };
             auto issue_SO = [&](int n) {  // S += K^T (D_hi + D_lo);  Y += M_hi D_hi + M_hi D_lo + M_lo D_hi
-                const uint32_t sa = stage_addr(n), yu = tmem + T_YU + 64 * (n & 1);
-                const uint32_t mhi = sbase + OFF_M + (n & 1) * 2 * SLOT, mlo = mhi + SLOT;
+                const uint32_t yu = tmem + T_YU + 64 * (n & 1);
+                const uint64_t dKt = sdesc_sw128(stage_addr(n) + SL_K0 * SLOT, BOXSTRIDE, 1024);
+                const uint64_t dM = sdesc_sw128(sbase + OFF_M + (n & 1) * 2 * SLOT, 16, 1024);
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + T_S, sdesc_sw128(sa + SL_K0 * SLOT + kk * 2048, BOXSTRIDE, 1024),
-                                 sdesc_sw128(dba + part * SLOT + kk * 2048, SLOT, 1024), ID_S, 1);
+                        mma_bf16(tmem + T_S, dKt + ((kk * 2048) >> 4), dDB + ((part * SLOT + kk * 2048) >> 4), ID_S, 1);
                 mma_commit(&bar[B_SFULL]);  // the state chain waits only for S
 #pragma unroll
                 for (int part = 0; part < 3; ++part) {
-                    const uint32_t ma = (part == 2) ? mlo : mhi, da = dba + (part == 1 ? SLOT : 0);
+                    const uint32_t moff = (part == 2) ? SLOT : 0, doff = (part == 1) ? SLOT : 0;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(yu, sdesc_sw128(ma + kk * 32, 16, 1024), sdesc_sw128(da + kk * 2048, SLOT, 1024),
-                                 ID_N64, 1);
+                        mma_bf16(yu, dM + ((moff + kk * 32) >> 4), dDB + ((doff + kk * 2048) >> 4), ID_N64, 1);
                 }
                 mma_commit(&bar[B_OFULL + (n & 1)]);
                 mma_commit(&bar[B_EMPTY + (n & 1)]);
@@ -597,8 +607,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             //   D(n)  after -W/M of chunk n (a2) and the bf16 state (sb);
             //   SO(n) after the bf16 D (delta);
             //   Y(m)  after X(m), after O(m-2) left the Y buffer (oread[m%2]) and
-            //         after D(m-1) was issued: D(m-1) waits for the -W readout
-            //         of chunk m-1, the last reader of the X K accumulator;
+            //         after D(m-2) was issued: D(m-2) waits for the -W readout
+            //         of chunk m-2, the last reader of X K buffer m%2;
             //   G(m)  after its TMA stage landed, G(m-1) was read (gempty) and
             //         SO(m-2) was issued (so the commit that signals G(m)
             //         also covers every earlier reader of the buffers that
@@ -618,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     EFLA_TR(21, nS); issue_SO(nS++);
                     did = true;
                 }
-                if (nY < nc && nY < nG && nY <= nD && mbar_test(&bar[B_XFULL], nY & 1) &&
+                if (nY < nc && nY < nG && nY <= nD + 1 && mbar_test(&bar[B_XFULL], nY & 1) &&
                     (nY < 2 || mbar_test(&bar[B_OREAD + (nY & 1)], ((nY - 2) >> 1) & 1))) {
                     tc_fence_after();
                     EFLA_TR(22, nY); issue_Y(nY++);
@@ -693,9 +703,11 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 
 constexpr int KLD = DK + 8;  // padded bf16 row stride of K: conflict-free mma.sync fragment loads
 struct TPrepSmem {
-    __nv_bfloat16 K[C][KLD];
+    union {  // K is dead once K K^T is formed; T reuses its space (6 CTAs per SM instead of 4)
+        __nv_bfloat16 K[C][KLD];
+        float T[C * LDF];
+    };
     float A[C * LDF];
-    float T[C * LDF];
     float alpha[C];
 };
 
