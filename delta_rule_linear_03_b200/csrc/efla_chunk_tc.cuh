@@ -6,38 +6,42 @@
 // flowchart) chunk by chunk in the UT form of the chunk-parallel scheme that
 // page cites (整体框架, "WY / UT"), with C = 64:
 //
-//   kernel chunk_T_kernel, one CTA per chunk, all chunks in parallel:
+//   kernel chunk_prep_kernel, one CTA per chunk, all chunks in parallel
+//   (everything that does not depend on the state):
 //   alpha = gate(beta, ||k||^2)                       (fp32, CUDA cores)
 //   A  = strictly-lower(diag(alpha) K K^T)            (mma.sync bf16, fp32 acc.)
-//   T  = (I + A)^{-1}                                 (CUDA cores + mma.sync TF32)
-//   X  = [0; T diag(alpha)]                           (bf16 hi + lo, to scratch)
+//   T  = (I + A)^{-1},  T' = T diag(alpha)            (CUDA cores + mma.sync TF32)
+//   M  = lower-incl-diag(Q K^T)                       (mma.sync bf16)
+//   W  = T' K,  U = T' V                              (mma.sync, T' as bf16 hi + lo)
+//   -> workspace: -W (bf16), M (bf16), U (fp32)
 //   kernel chunk_tc_kernel, serial over the chunks of one (b, h, d_v half):
-//   G  = [K; Q] K^T                                   (tcgen05, M=128 N=64 K=128)
-//   [. ; W] = X K,   [0; U] = X V_tile                (tcgen05, N=128 and N=64)
-//   Y += [Q; -W] S  ->  [Q S; U - W S] = [Q S; D]     (tcgen05, N=64 K=128)
+//   Y  = [Q; -W] S          ->  [Q S; -W S]           (tcgen05, M=128 N=64 K=128)
+//   D  = U + (-W S)                                   (CUDA cores, TMEM -> smem)
 //   S += K^T D                                        (tcgen05, N=64 K=64)
-//   Y += [M; *] D   ->  O = Q S + M D,  M = lower-incl-diag(Q K^T)
+//   Y += [M; *] D           ->  O = Q S + M D         (tcgen05, N=64 K=64)
 //
 // Every product is stacked to M = 128 rows so the accumulator of each
 // tcgen05.mma occupies all 128 TMEM lanes, one row per lane.  (In the last
 // product the lower 64 rows of the A operand are whatever follows M in shared
-// memory: they only add into the D rows of Y, which are dead by then.)
+// memory: they only add into the -W S rows of Y, which are dead by then.)
 //
-// Precision: q, k, v are exact bf16 operands.  T diag(alpha), S, D and M are
-// fp32 values fed to the bf16 tensor cores as a hi + lo pair of bf16
-// (x = hi + lo to ~16 significant bits); only -W goes in as a single bf16.
-// Accumulation is fp32 in TMEM and the state is kept in fp32.
+// Precision: q, k, v are exact bf16 operands.  S, D and T' are fp32 values
+// fed to the bf16 tensor cores as a hi + lo pair of bf16 (x = hi + lo to ~16
+// significant bits); -W and M go in as single bf16 (M only reaches the
+// output, not the state).  Accumulation is fp32 (TMEM or mma.sync registers)
+// and the state is kept in fp32.
 //
-// Everything S-independent and per-chunk that is not a tensor-core product
-// (the gate and T) runs in the first kernel, so the serial kernel only moves
-// T' in and keeps its tensor pipe and state chain busy.
+// The serial kernel holds only the state chain Y -> D -> S and the output
+// product, so its tensor pipe is never busy with work the chain waits behind.
 // One CTA per (b, h, half of d_v): the 128 x 64 fp32 state tile lives in
 // TMEM for the whole sequence.  Warp roles:
-//   warps 0-1  "io":    T' image in (chunk n+1), O of chunk n-1 out to HBM
-//   warps 2-3  "mw":    M and -W for chunk n+1 (S-independent)
-//   warps 4-7  "state": D -> bf16 and S -> bf16 for chunk n (the serial chain)
+//   warps 0-7  TMEM <-> registers <-> smem, each warp a 32-lane x 32-column
+//              quarter-half: all 8 read S (-> bf16 hi/lo operand); warps
+//              2,3,6,7 (lanes 64..127) form D; warps 0,1,4,5 (lanes 0..63)
+//              read O out to HBM
 //   warp 8     one thread issues every tcgen05.mma and commit
-//   warp 9     one thread issues the TMA loads (2-stage K/Q/V ring)
+//   warp 9     one thread issues the TMA loads (2-stage ring: Q, K tiles and
+//              the -W, M, U images of the workspace)
 // Every mbarrier wait is bounded; a wait that gives up sets the sticky
 // device error word and an abort flag, every role then leaves its loop, the
 // MMA thread drains its outstanding MMAs and the TMA thread its copies, and
@@ -56,53 +60,55 @@ namespace tc {
 
 constexpr int C = 64, DK = 128, DVT = 64, NSPLIT = 2;
 constexpr int kThreads = 320;
-constexpr uint32_t SLOT = 8192;                 // one 64 x 64 bf16 swizzled box
-constexpr uint32_t STAGE = 7 * SLOT;            // K0 Q0 W0 K1 Q1 W1 V
-constexpr uint32_t SL_K0 = 0, SL_Q0 = 1, SL_W0 = 2, SL_V = 6;
-constexpr uint32_t BOXSTRIDE = 3 * SLOT;        // K0->K1, Q0->Q1, W0->W1
-constexpr int LDF = 64;                         // fp32 row stride of A and T
-constexpr uint32_t OFF_M = 2 * STAGE;           // M hi/lo for chunk parity 0 and 1: 4 boxes
-constexpr uint32_t OFF_Z0 = OFF_M + 4 * SLOT;   // zero box, then T' hi  ([0; T'hi] operand)
-constexpr uint32_t OFF_THI = OFF_Z0 + SLOT;
-constexpr uint32_t OFF_Z1 = OFF_THI + SLOT;     // zero box, then T' lo  ([0; T'lo] operand)
-constexpr uint32_t OFF_TLO = OFF_Z1 + SLOT;
-constexpr uint32_t OFF_SB = OFF_TLO + SLOT;     // S tile bf16 hi, then lo (MN-major B), 128 x 64 each
-constexpr uint32_t OFF_DB = OFF_SB + 4 * SLOT;  // D bf16 hi, then lo (MN-major B), 64 x 64 each
-constexpr uint32_t OFF_BAR = OFF_DB + 2 * SLOT;
-constexpr uint32_t XBYTES = 2 * SLOT;           // T' hi and lo boxes of one chunk (workspace image)
-constexpr uint32_t NBAR = 20;  // indices 0..19
+constexpr uint32_t SLOT = 8192;  // one 64 x 64 bf16 swizzled box
+// Per-chunk workspace image written by chunk_prep_kernel:
+//   [0, 16K)   -W, two boxes (d_k columns 0-63, 64-127), 128-byte swizzle
+//   [16K, 24K) M box, 128-byte swizzle
+//   [24K, 56K) U fp32, two d_v halves of 64 rows x 256 B; the 16-byte
+//              chunk j of row r sits at position j ^ (r & 15)
+constexpr uint32_t IMG_W = 0, IMG_M = 2 * SLOT, IMG_U = 3 * SLOT, PREP_BYTES = 7 * SLOT;
+constexpr uint32_t UHALF = 2 * SLOT;
+// Shared-memory stage (one chunk), in 8 KB slots: Q0 W0 Q1 W1 K0 K1 M U U.
+// [Q0; W0] and [Q1; W1] are the two K-halves of the 128-row A operand [Q; -W].
+constexpr uint32_t SL_Q0 = 0, SL_W0 = 1, SL_K0 = 4, SL_M = 6, SL_U = 7, NSLOTS = 9;
+constexpr uint32_t STAGE = NSLOTS * SLOT;
+// A stage lands in two parts with their own barriers: part A (Q, -W), read by
+// Y = [Q; -W] S only, and part B (K, M, U), read until the end of the chunk;
+// part A of chunk n+2 can then load as soon as Y of chunk n is done.
+constexpr uint32_t TX_A = 4 * SLOT, TX_B = 5 * SLOT;
+static_assert(TX_A + TX_B == STAGE, "stage parts");
+constexpr int LDF = 64;                          // fp32 row stride of A and T (prep)
+constexpr uint32_t OFF_SB = 2 * STAGE;           // S tile bf16 hi, then lo (MN-major B), 128 x 64 each
+constexpr uint32_t OFF_DB = OFF_SB + 4 * SLOT;   // [2] D bf16 hi, then lo (MN-major B), 64 x 64 each
+constexpr uint32_t OFF_OST = OFF_DB + 4 * SLOT;  // O tile staged for the TMA store (64 x 64, fp32 or bf16)
+constexpr uint32_t OFF_BAR = OFF_OST + 2 * SLOT;
+constexpr uint32_t NBAR = 20;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
-// TMEM columns (fp32, 128 lanes)
-// X K accumulates into two alternating buffers (YW, by chunk parity) so
-// Y(n+1) can run while the -W readout of chunk n is still pending.
-constexpr uint32_t T_S = 0, T_G = 64, T_YW = 128, T_YU = 384, TMEM_COLS = 512;
+// TMEM columns (fp32, 128 lanes): the state tile, then two Y accumulators
+// (by chunk parity) so O of chunk n can wait in TMEM while Y(n+1) runs.
+constexpr uint32_t T_S = 0, T_Y = 64, TMEM_COLS = 256;
 
 enum : int {
-    B_FULL = 0,     // [2] TMA stage landed
-    B_EMPTY = 2,    // [2] stage free again (commit after the last MMA reading it)
-    B_GFULL = 4,    // G ready in TMEM
-    B_GEMPTY = 5,   // G read out
-    B_XFULL = 6,    // T' image of the next chunk in place
-    B_YFULL = 7,    // [2] X K and X V of a chunk done (per X K buffer)
-    B_A2FULL = 9,   // [2] -W and M written for chunk parity b
-    B_SBFULL = 11,  // bf16 S tile written
-    B_DFULL = 12,   // Y += [Q;-W] S done
-    B_DELTA = 13,   // bf16 D written
-    B_SFULL = 14,   // S += K^T D done
-    B_DRAIN = 15,   // final drain of the MMA pipe
-    B_OREAD = 16,   // [2] O of a chunk read out of Y buffer b
-    B_OFULL = 18,   // [2] O += M D done for Y buffer b
+    B_FULLA = 0,    // [2] stage part A landed (TMA transaction count)
+    B_FULLB = 2,    // [2] stage part B landed
+    B_EMPTYA = 4,   // [2] part A free again (commit after Y)
+    B_EMPTYB = 6,   // [2] part B free again (commit after O)
+    B_SBFULL = 8,   // bf16 S tile written (256 threads)
+    B_DFULL = 9,    // Y = [Q; -W] S done
+    B_DELTA = 10,   // bf16 D written (128 threads)
+    B_SFULL = 11,   // S += K^T D done
+    B_DRAIN = 12,   // final drain of the MMA pipe
+    B_OREAD = 13,   // [2] O of a chunk read out of Y buffer b (128 threads)
+    B_OFULL = 15,   // [2] O += M D done for Y buffer b
 };
 // Barriers that complete once per chunk but can be waited on a chunk late
 // come in pairs indexed by chunk parity: each then completes once per two
 // chunks, so a parity wait can never see it two phases ahead.
 
-constexpr uint32_t ID_G = ptx::idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_YW = ptx::idesc_bf16(128, 128, false, true);
-constexpr uint32_t ID_N64 = ptx::idesc_bf16(128, 64, false, true);
+constexpr uint32_t ID_Y = ptx::idesc_bf16(128, 64, false, true);
 constexpr uint32_t ID_S = ptx::idesc_bf16(128, 64, true, true);
 
 // Optional timeline trace (compile with -DEFLA_TRACE): threads of CTA 0
@@ -171,15 +177,18 @@ struct Split64 {
 };
 
 // T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A.  First the
-// four 16 x 16 diagonal blocks by right-looking forward substitution (one
-// warp per block, one column per lane pair, fp32); then block rows I = 1..3:
+// four 16 x 16 diagonal blocks by right-looking forward substitution (warps
+// 0-3, one block each, one column per lane pair, fp32); then block rows
+// I = 1..3:
 //     R = A_{I,<I} T_{<I,<I},   T_{I,<I} = -T_II R,
 // as 16 x 8 tiles on mma.sync (TF32 operands, fp32 accumulation).  TF32
 // here costs nothing measurable: T then feeds bf16 hi/lo operands, and an
-// emulation of the whole kernel gave the same error against the oracle
-// with fp32 or TF32 block products.  128 threads (prep).
-__device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af, const Split64 Tf, int n_trace = 0) {
-    {
+// emulation of the whole computation gave the same error against the
+// oracle with fp32 or TF32 block products.  NT threads (a multiple of 128)
+// call it together; it ends with all of them synchronised on barrier 1.
+template <int NT>
+__device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af, const Split64 Tf) {
+    if (p < 128) {
         const int w = p >> 5, l = p & 31, c = l & 15, h = l >> 4, base = 16 * w;
         float acc[8];
 #pragma unroll
@@ -192,19 +201,18 @@ __device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af,
         }
 #pragma unroll
         for (int s = 0; s < 8; ++s) *Tf.at(base + 2 * s + h, base + c) = acc[s];
-        if (l == 0) EFLA_TR(30 + w, n_trace);
     }
-    ptx::named_bar(1, 128);
+    ptx::named_bar(1, NT);
     // Block rows on the tensor cores through mma.sync m16n8k8 (TF32 inputs,
-    // fp32 accumulation): warp w owns the 8-column tiles jt = w, w+4, ... of
-    // block row I, so R's tile and the T tile computed from it stay inside
+    // fp32 accumulation): warp w owns the 8-column tiles jt = w, w + NT/32, ...
+    // of block row I, so R's tile and the T tile computed from it stay inside
     // one warp.  R is parked in T's own slots between the two products.
     const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll 1
     for (int I = 1; I < 4; ++I) {
         const int r0 = 16 * I;
 #pragma unroll 1
-        for (int jt = w; jt < 2 * I; jt += 4) {
+        for (int jt = w; jt < 2 * I; jt += NT / 32) {
             const int c0 = 8 * jt;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             // R tile = A[r0.., k] T[k, c0..] over k from the column's own block up to r0
@@ -240,15 +248,9 @@ __device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af,
             *Tf.at(r0 + g + 8, c0 + 2 * t) = -out[2];
             *Tf.at(r0 + g + 8, c0 + 2 * t + 1) = -out[3];
         }
-        if (lane == 0) EFLA_TR(40 + 4 * I + w, n_trace);
-        ptx::named_bar(1, 128);
+        ptx::named_bar(1, NT);
     }
 }
-
-// One 64-value fp32 row (held as two 32-register halves) -> bf16 hi at
-// `base` and lo at `base + lo_off`, row `row` of a 128-byte-swizzled tile.
-__device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo_off, int row, const uint32_t (&a)[32],
-                                                const uint32_t (&b)[32]);
 
 // bf16 hi + lo split of a pair of fp32 values (hi = rn(x), lo = rn(x - hi)).
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
@@ -260,28 +262,59 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_
     lo = l;
 }
 
-__device__ __forceinline__ void write_split_row(unsigned char *base, uint32_t lo_off, int row, const uint32_t (&a)[32],
-                                                const uint32_t (&b)[32]) {
+// 32 fp32 values (columns 8 * chunk0 ..) of row `row` -> bf16 hi at `base`
+// and lo at `base + lo_off`, in a 128-byte-swizzled tile of 64-column rows.
+__device__ __forceinline__ void write_split32(unsigned char *base, uint32_t lo_off, int row, int chunk0,
+                                              const float (&x)[32]) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
         uint32_t h4[4], l4[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int c0 = 8 * j + 2 * u;
-            const float x0 = __uint_as_float(c0 < 32 ? a[c0] : b[c0 - 32]);
-            const float x1 = __uint_as_float(c0 + 1 < 32 ? a[c0 + 1] : b[c0 + 1 - 32]);
-            split2(x0, x1, h4[u], l4[u]);
-        }
-        *reinterpret_cast<uint4 *>(base + ptx::sw128_chunk(row, j)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-        *reinterpret_cast<uint4 *>(base + lo_off + ptx::sw128_chunk(row, j)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+        for (int u = 0; u < 4; ++u) split2(x[8 * j + 2 * u], x[8 * j + 2 * u + 1], h4[u], l4[u]);
+        const uint32_t off = ptx::sw128_chunk(row, chunk0 + j);
+        *reinterpret_cast<uint4 *>(base + off) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+        *reinterpret_cast<uint4 *>(base + lo_off + off) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
     }
+}
+
+__device__ __forceinline__ void as_float32(const uint32_t (&r)[32], float (&x)[32]) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+}
+
+// cp.async.bulk global -> shared, `bytes` (multiple of 16, both ends 16-byte
+// aligned), completing as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            ptx::smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(ptx::smem_u32(bar))
+        : "memory");
+}
+
+// TMA tensor store of one box from shared memory (bulk async group of this thread).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(ptx::smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Bounded wait by a whole warp; the answer is warp-uniform (false when any lane gave up).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort));
 }
 
 template <typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const unsigned char *__restrict__ xws,
-                    const float *__restrict__ S0, Tout *__restrict__ o, float *__restrict__ SL, int L, int nc) {
+                    const __grid_constant__ CUtensorMap tm_o, const unsigned char *__restrict__ ws,
+                    const float *__restrict__ S0, float *__restrict__ SL, int L, int nc) {
     using namespace ptx;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
@@ -293,396 +326,305 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long bh = blockIdx.x / NSPLIT;
-    const int j0 = (blockIdx.x % NSPLIT) * DVT;
+    const int half = blockIdx.x % NSPLIT, j0 = half * DVT;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        mbar_init(&bar[B_FULL], 1);
-        mbar_init(&bar[B_FULL + 1], 1);
-        mbar_init(&bar[B_EMPTY], 1);
-        mbar_init(&bar[B_EMPTY + 1], 1);
-        mbar_init(&bar[B_GFULL], 1);
-        mbar_init(&bar[B_GEMPTY], 64);
-        mbar_init(&bar[B_XFULL], 64);
-        mbar_init(&bar[B_YFULL], 1);
-        mbar_init(&bar[B_YFULL + 1], 1);
-        mbar_init(&bar[B_A2FULL], 64);
-        mbar_init(&bar[B_A2FULL + 1], 64);
-        mbar_init(&bar[B_SBFULL], 128);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[B_FULLA + s], 1);
+            mbar_init(&bar[B_FULLB + s], 1);
+            mbar_init(&bar[B_EMPTYA + s], 1);
+            mbar_init(&bar[B_EMPTYB + s], 1);
+            mbar_init(&bar[B_OREAD + s], 128);
+            mbar_init(&bar[B_OFULL + s], 1);
+        }
+        mbar_init(&bar[B_SBFULL], 256);
         mbar_init(&bar[B_DFULL], 1);
         mbar_init(&bar[B_DELTA], 128);
         mbar_init(&bar[B_SFULL], 1);
         mbar_init(&bar[B_DRAIN], 1);
-        mbar_init(&bar[B_OREAD], 64);
-        mbar_init(&bar[B_OREAD + 1], 64);
-        mbar_init(&bar[B_OFULL], 1);
-        mbar_init(&bar[B_OFULL + 1], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
-    // constant zero boxes: rows 0-63 of the [0; T' hi] and [0; T' lo] operands
-    for (int i = threadIdx.x; i < 2 * (int)SLOT / 16; i += kThreads) {
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4 *>(sm + (i < (int)SLOT / 16 ? OFF_Z0 : OFF_Z1 - SLOT) + 16 * i) = z;
-    }
-    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp < 2) {
-        // ------------------------------------------------------------ io (warps 0-1)
-        // T' = T diag(alpha) of every chunk arrives precomputed from
-        // chunk_T_kernel as hi and lo bf16 boxes, already in the swizzled
-        // image the X operand descriptors read: copy it in (prefetched a
-        // chunk ahead in registers).  Then read O of the previous chunk out
-        // of TMEM lanes 0..63 and store it.
-        const int p = threadIdx.x;  // TMEM lane / chunk row
-        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
-        const uint4 *xsrc = reinterpret_cast<const uint4 *>(xws + (size_t)bh * nc * XBYTES);
-        uint4 xr[16];
+    if (warp < 8) {
+        // ------------------------------------------------------------ TMEM <-> smem warps
+        // Warp w owns TMEM lanes 32 (w % 4) .. + 31 and columns 32 (w / 4) .. + 31
+        // of every 64-column tile.
+        const int quad = warp & 3, cpart = warp >> 2, c0 = 32 * cpart;
+        const int row = 32 * quad + lane;  // TMEM lane: state row, or chunk row (+64 for D)
+        const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
+        const bool dwarp = quad >= 2;  // lanes 64..127: the D rows of Y
+        float x[32];
+        {   // initial state
+            const float *src = S0 ? S0 + ((size_t)bh * DK + row) * DK + j0 + c0 : nullptr;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) xr[i] = __ldcs(xsrc + p + 64 * i);
-        auto read_O = [&](int m) -> bool {
-            const bool ok = mbar_wait(&bar[B_OFULL + (m & 1)], (m >> 1) & 1, abort_flag);
-            if (bar_any(3, 64, !ok || *abort_flag)) return false;
-            tc_fence_after();
-            uint32_t oa[32], ob[32];
-            tmem_ld32(tl + T_YU + 64 * (m & 1), oa);
-            tmem_ld32(tl + T_YU + 64 * (m & 1) + 32, ob);
-            tmem_ld_wait(oa);
-            tmem_ld_wait(ob);
-            tc_fence_before();
-            mbar_arrive(&bar[B_OREAD + (m & 1)]);
-            if (p == 0) EFLA_TR(14, m);
-            if (m * C + p < L) {
-                Tout *dst = o + ((size_t)bh * L + m * C + p) * DK + j0;
-#pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    const uint32_t *src = (c < 32) ? &oa[c] : &ob[c - 32];
-                    store4(dst + c, make_float4(__uint_as_float(src[0]), __uint_as_float(src[1]),
-                                                __uint_as_float(src[2]), __uint_as_float(src[3])));
-                }
-            }
-            return true;
-        };
-        bool alive = true;
-        for (int n = 0; n < nc && alive; ++n) {
-            if (n > 0) {  // the [0; T'] boxes are free once Y(n-1) completed
-                const bool ok = mbar_wait(&bar[B_YFULL + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_flag);
-                if (bar_any(3, 64, !ok || *abort_flag)) break;
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const uint32_t bo = 16u * (uint32_t)(p + 64 * i);  // byte offset in the 16 KB image
-                *reinterpret_cast<uint4 *>(sm + (bo < SLOT ? OFF_THI + bo : OFF_TLO + (bo - SLOT))) = xr[i];
-            }
-            fence_proxy_async();
-            mbar_arrive(&bar[B_XFULL]);
-            if (p == 0) EFLA_TR(5, n);
-            if (n + 1 < nc) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) xr[i] = __ldcs(xsrc + (size_t)(n + 1) * (XBYTES / 16) + p + 64 * i);
-            }
-            if (n > 0) alive = read_O(n - 1);
-        }
-        if (alive && !*abort_flag) read_O(nc - 1);
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ mw (warps 2-3)
-        // M = lower(Q K^T) as hi/lo boxes and -W from X K; both live in TMEM
-        // lanes 64..127, which these warps own.
-        const int r = threadIdx.x - 64;  // chunk row
-        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
-        for (int n = 0; n < nc; ++n) {
-            unsigned char *st = sm + (n & 1) * STAGE;
-            bool ok = mbar_wait(&bar[B_GFULL], n & 1, abort_flag);
-            if (r == 0) EFLA_TR(2, n);
-            if (bar_any(1, 64, !ok || *abort_flag)) break;
-            tc_fence_after();
-            {
-                uint32_t ga[32], gb[32];
-                tmem_ld32(tl + T_G, ga);
-                tmem_ld32(tl + T_G + 32, gb);
-                tmem_ld_wait(ga);
-                tmem_ld_wait(gb);
-                tc_fence_before();
-                mbar_arrive(&bar[B_GEMPTY]);
-                unsigned char *mhi = sm + OFF_M + (n & 1) * 2 * SLOT, *mlo = mhi + SLOT;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    uint32_t h4[4], l4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c0 = 8 * j + 2 * e;
-                        const float x0 = (c0 <= r) ? __uint_as_float(c0 < 32 ? ga[c0] : gb[c0 - 32]) : 0.f;
-                        const float x1 =
-                            (c0 + 1 <= r) ? __uint_as_float(c0 + 1 < 32 ? ga[c0 + 1] : gb[c0 + 1 - 32]) : 0.f;
-                        split2(x0, x1, h4[e], l4[e]);
-                    }
-                    *reinterpret_cast<uint4 *>(mhi + sw128_chunk(r, j)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-                    *reinterpret_cast<uint4 *>(mlo + sw128_chunk(r, j)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
-                }
-            }
-            if (r == 0) EFLA_TR(3, n);
-            ok = mbar_wait(&bar[B_YFULL + (n & 1)], (n >> 1) & 1, abort_flag);
-            if (r == 0) EFLA_TR(6, n);
-            if (bar_any(1, 64, !ok || *abort_flag)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t wa[32], wb[32];
-                tmem_ld32(tl + T_YW + 128 * (n & 1) + 64 * h, wa);
-                tmem_ld32(tl + T_YW + 128 * (n & 1) + 64 * h + 32, wb);
-                tmem_ld_wait(wa);
-                tmem_ld_wait(wb);
-                unsigned char *wrow = st + SL_W0 * SLOT + h * BOXSTRIDE;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c0 = 8 * j + 2 * u;
-                        const float x0 = __uint_as_float(c0 < 32 ? wa[c0] : wb[c0 - 32]);
-                        const float x1 = __uint_as_float(c0 + 1 < 32 ? wa[c0 + 1] : wb[c0 + 1 - 32]);
-                        w4[u] = pack_bf16(-x0, -x1);
-                    }
-                    *reinterpret_cast<uint4 *>(wrow + sw128_chunk(r, j)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                }
-            }
-            fence_proxy_async();
-            tc_fence_before();
-            mbar_arrive(&bar[B_A2FULL + (n & 1)]);
-            if (r == 0) EFLA_TR(7, n);
-        }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ state
-        const int q = threadIdx.x - 128;  // TMEM lane / state row
-        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        {
-            uint32_t ra[32], rb[32];
-            const float *src = S0 ? S0 + ((size_t)bh * DK + q) * DK + j0 : nullptr;
-#pragma unroll
-            for (int c = 0; c < 64; c += 4) {
+            for (int c = 0; c < 32; c += 4) {
                 const float4 v = src ? *reinterpret_cast<const float4 *>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-                uint32_t *dst = (c < 32) ? &ra[c] : &rb[c - 32];
-                dst[0] = __float_as_uint(v.x);
-                dst[1] = __float_as_uint(v.y);
-                dst[2] = __float_as_uint(v.z);
-                dst[3] = __float_as_uint(v.w);
+                x[c] = v.x;
+                x[c + 1] = v.y;
+                x[c + 2] = v.z;
+                x[c + 3] = v.w;
             }
-            tmem_st32(tl + T_S, ra);
-            tmem_st32(tl + T_S + 32, rb);
+            uint32_t r[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
+            tmem_st32(tl + T_S + c0, r);
             tmem_st_wait();
-            write_split_row(sm + OFF_SB, 2 * SLOT, q, ra, rb);
+            write_split32(sm + OFF_SB, 2 * SLOT, row, 4 * cpart, x);
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bar[B_SBFULL]);
         }
+        // Only the 256-thread vote on barrier 2 leaves the loop: a failed wait
+        // inside one group (barriers 1 and 3) skips that group's work, and the
+        // abort flag it set makes the next vote leave.
         for (int n = 0; n < nc; ++n) {
             const int b = n & 1;
-            bool ok = mbar_wait(&bar[B_DFULL], n & 1, abort_flag);
-            if (q == 64) EFLA_TR(10, n);
-            if (bar_any(2, 128, !ok || *abort_flag)) break;
-            tc_fence_after();
-            if (warp >= 6) {  // D rows (lanes 64..127) -> bf16 MN-major operand, row c = lane - 64
-                const int c = q - 64;
-                uint32_t da[32], db[32];
-                tmem_ld32(tl + T_YU + 64 * b, da);
-                tmem_ld32(tl + T_YU + 64 * b + 32, db);
-                tmem_ld_wait(da);
-                tmem_ld_wait(db);
-                if (q == 64) EFLA_TR(15, n);
-                write_split_row(sm + OFF_DB, SLOT, c, da, db);
-                if (q == 64) EFLA_TR(16, n);
-            }
-            fence_proxy_async();
-            if (q == 64) EFLA_TR(17, n);
-            tc_fence_before();
-            mbar_arrive(&bar[B_DELTA]);
-            if (q == 64) EFLA_TR(11, n);
-            ok = mbar_wait(&bar[B_SFULL], n & 1, abort_flag);
-            if (q == 64) EFLA_TR(12, n);
-            if (bar_any(2, 128, !ok || *abort_flag)) break;
-            tc_fence_after();
-            uint32_t sa[32], sb[32];
-            tmem_ld32(tl + T_S, sa);
-            tmem_ld32(tl + T_S + 32, sb);
-            tmem_ld_wait(sa);
-            tmem_ld_wait(sb);
-            if (q == 64) EFLA_TR(24, n);
-            write_split_row(sm + OFF_SB, 2 * SLOT, q, sa, sb);
-            if (q == 64) EFLA_TR(25, n);
-            fence_proxy_async();
-            tc_fence_before();
-            mbar_arrive(&bar[B_SBFULL]);
-            if (q == 64) EFLA_TR(13, n);
-            if (n == nc - 1 && SL) {
-                float *dst = SL + ((size_t)bh * DK + q) * DK + j0;
+            const uint32_t ty = T_Y + 64 * b + c0;
+            bool bad = false;
+            if (dwarp) {
+                // D = U + (-W S): TMEM lanes 64..127 of Y, plus U from the stage
+                const int c = row - 64;
+                // (the stage's own barrier too: U landed by the bulk copy is
+                // visible to the threads that observe that barrier's phase)
+                bool ok = mbar_wait(&bar[B_DFULL], n & 1, abort_flag);
+                if (row == 64 && cpart == 0) EFLA_TR(28, n);
+                ok = ok && mbar_wait(&bar[B_FULLB + b], (n >> 1) & 1, abort_flag);
+                if (row == 64 && cpart == 0) EFLA_TR(10, n);
+                bad = bar_any(1, 128, !ok || *abort_flag);
+                if (!bad) {
+                    tc_fence_after();
+                    uint32_t r[32];
+                    tmem_ld32(tl + ty, r);
+                    const unsigned char *urow = sm + b * STAGE + SL_U * SLOT + c * 256;
+                    float u[32];
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    const uint32_t *src = (c < 32) ? &sa[c] : &sb[c - 32];
-                    *reinterpret_cast<float4 *>(dst + c) = make_float4(
-                        __uint_as_float(src[0]), __uint_as_float(src[1]), __uint_as_float(src[2]),
-                        __uint_as_float(src[3]));
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 v =
+                            *reinterpret_cast<const float4 *>(urow + (((uint32_t)(8 * cpart + j) ^ (c & 15)) << 4));
+                        u[4 * j] = v.x;
+                        u[4 * j + 1] = v.y;
+                        u[4 * j + 2] = v.z;
+                        u[4 * j + 3] = v.w;
+                    }
+                    tmem_ld_wait(r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = u[i] + __uint_as_float(r[i]);
+                    write_split32(sm + OFF_DB + b * 2 * SLOT, SLOT, c, 4 * cpart, x);
+                    fence_proxy_async();
+                    tc_fence_before();
+                    mbar_arrive(&bar[B_DELTA]);
+                    if (row == 64 && cpart == 0) EFLA_TR(11, n);
+                }
+            }
+            const bool ok = !bad && mbar_wait(&bar[B_SFULL], n & 1, abort_flag);
+            if (row == 64 && cpart == 0) EFLA_TR(12, n);
+            if (bar_any(2, 256, !ok || *abort_flag)) break;
+            if (row == 64 && cpart == 0) EFLA_TR(29, n);
+            tc_fence_after();
+            {
+                uint32_t r[32];
+                tmem_ld32(tl + T_S + c0, r);
+                tmem_ld_wait(r);
+                if (row == 64 && cpart == 0) EFLA_TR(30, n);
+                as_float32(r, x);
+                write_split32(sm + OFF_SB, 2 * SLOT, row, 4 * cpart, x);
+                if (row == 64 && cpart == 0) EFLA_TR(31, n);
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(&bar[B_SBFULL]);
+                if (row == 64 && cpart == 0) EFLA_TR(13, n);
+            }
+            if (n == nc - 1 && SL) {
+                float *dst = SL + ((size_t)bh * DK + row) * DK + j0 + c0;
+#pragma unroll
+                for (int c = 0; c < 32; c += 4)
+                    *reinterpret_cast<float4 *>(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+            }
+            if (!dwarp) {
+                // O = Q S + M D: TMEM lanes 0..63 of Y -> staging tile -> one TMA
+                // store (rows past L are clipped by the tensor map).  The staging
+                // tile is rewritten only after the previous store has read it.
+                const bool storer = warp == 0 && lane == 0;
+                const bool okO = mbar_wait(&bar[B_OFULL + b], (n >> 1) & 1, abort_flag);
+                if (storer) bulk_wait_read0();
+                if (!bar_any(3, 128, !okO || *abort_flag)) {
+                    tc_fence_after();
+                    uint32_t r[32];
+                    tmem_ld32(tl + ty, r);
+                    tmem_ld_wait(r);
+                    tc_fence_before();
+                    mbar_arrive(&bar[B_OREAD + b]);
+                    if (row == 0 && cpart == 0) EFLA_TR(14, n);
+                    // staging: 128-byte-swizzled boxes of 128-byte rows -- fp32: two
+                    // 32-column boxes (one per column half c0); bf16: one 64-column box
+                    if constexpr (sizeof(Tout) == 4) {
+                        unsigned char *orow = sm + OFF_OST + cpart * SLOT + row * 128;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            *reinterpret_cast<uint4 *>(orow + ((i ^ (row & 7)) << 4)) =
+                                make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+                    } else {
+                        unsigned char *orow = sm + OFF_OST + row * 128;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float *f = reinterpret_cast<const float *>(&r[8 * i]);
+                            *reinterpret_cast<uint4 *>(orow + (((4 * cpart + i) ^ (row & 7)) << 4)) =
+                                make_uint4(ptx::pack_bf16(f[0], f[1]), ptx::pack_bf16(f[2], f[3]),
+                                           ptx::pack_bf16(f[4], f[5]), ptx::pack_bf16(f[6], f[7]));
+                        }
+                    }
+                    fence_proxy_async();
+                    named_bar(3, 128);
+                    if (storer) {
+                        tma_store_3d(&tm_o, sm + OFF_OST, j0, n * C, (int)bh);
+                        if constexpr (sizeof(Tout) == 4) tma_store_3d(&tm_o, sm + OFF_OST + SLOT, j0 + 32, n * C, (int)bh);
+                        bulk_commit();
+                    }
                 }
             }
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t sba = sbase + OFF_SB, dba = sbase + OFF_DB;
-            const uint32_t xhi = sbase + OFF_Z0, xlo = sbase + OFF_Z1;  // [0; T' hi], [0; T' lo]
-            auto stage_addr = [&](int n) { return sbase + (uint32_t)(n & 1) * STAGE; };
-            // Descriptors: the 14-bit start-address field holds addr >> 4, and
-            // shared addresses stay below 256 KB, so the field never carries:
-            // the descriptor of (addr + off) is desc(addr) + (off >> 4).  Each group
-            // builds its base descriptors once; the unrolled k-steps add
-            // compile-time offsets, keeping the single issuing thread ahead of
-            // the tensor pipe.
-            const uint64_t dX[2] = {sdesc_sw128(xhi, 16, 1024), sdesc_sw128(xlo, 16, 1024)};
-            const uint64_t dSB = sdesc_sw128(sba, SLOT, 1024), dDB = sdesc_sw128(dba, SLOT, 1024);
-            auto issue_G = [&](int n) {
-                const uint64_t d0 = sdesc_sw128(stage_addr(n) + SL_K0 * SLOT, 16, 1024);
+        // The whole warp runs the loop and waits (a lone lane waiting while
+        // its 31 siblings sit at a convergence point notices completed
+        // barrier phases late); lane 0 issues every tcgen05.mma and commit.
+        // Descriptors: the 14-bit start-address field holds addr >> 4, and
+        // shared addresses stay below 256 KB, so the field never carries: the
+        // descriptor of (addr + off) is desc(addr) + (off >> 4).  Each product
+        // builds its base descriptors once; the unrolled k-steps add
+        // compile-time offsets, keeping the issuing lane ahead of the pipe.
+        const bool leader = lane == 0;
+        const uint64_t dSB = sdesc_sw128(sbase + OFF_SB, SLOT, 1024);
+        const uint64_t dDB = sdesc_sw128(sbase + OFF_DB, SLOT, 1024);
+        // O += M (D_hi + D_lo) of chunk m: issued behind Y of chunk m+1, so it
+        // runs while the state warps convert D of chunk m+1 (its readers then
+        // wait a little longer, the state chain does not).
+        auto issue_O = [&](int m) {
+            const int b = m & 1;
+            const uint64_t dM = sdesc_sw128(sbase + (uint32_t)b * STAGE + SL_M * SLOT, 16, 1024);
+            const uint64_t dD = dDB + ((b * 2 * SLOT) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t d = d0 + (((kk >> 2) * BOXSTRIDE + (kk & 3) * 32) >> 4);
-                    mma_bf16(tmem + T_G, d, d, ID_G, kk > 0);
-                }
-                mma_commit(&bar[B_GFULL]);
-            };
-            auto issue_Y = [&](int n) {  // Y = X_hi [K | V] + X_lo [K | V]
-                const uint32_t sa = stage_addr(n), yu = tmem + T_YU + 64 * (n & 1);
-                const uint64_t dK = sdesc_sw128(sa + SL_K0 * SLOT, BOXSTRIDE, 1024);
-                const uint64_t dV = sdesc_sw128(sa + SL_V * SLOT, SLOT, 1024);
+            for (int part = 0; part < 2; ++part)
 #pragma unroll
-                for (int part = 0; part < 2; ++part) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + T_YW + 128 * (n & 1), dX[part] + ((kk * 32) >> 4), dK + ((kk * 2048) >> 4),
-                                 ID_YW, part | kk);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(yu, dX[part] + ((kk * 32) >> 4), dV + ((kk * 2048) >> 4), ID_N64, part | kk);
-                }
-                mma_commit(&bar[B_YFULL + (n & 1)]);
-            };
-            auto issue_D = [&](int n) {  // Y += [Q; -W] (S_hi + S_lo)
-                const uint32_t yu = tmem + T_YU + 64 * (n & 1);
-                const uint64_t dA = sdesc_sw128(stage_addr(n) + SL_Q0 * SLOT, 16, 1024);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + T_Y + 64 * b, dM + ((kk * 32) >> 4), dD + ((part * SLOT + kk * 2048) >> 4), ID_Y, 1);
+            mma_commit(&bar[B_OFULL + b]);
+            mma_commit(&bar[B_EMPTYB + b]);
+        };
+        int n = 0;
+        for (; n < nc; ++n) {
+            const int s = n & 1;
+            const uint32_t sa = sbase + (uint32_t)s * STAGE, ty = tmem + T_Y + 64 * s;
+            // Y = [Q; -W] (S_hi + S_lo) after: part A of the stage landed, O of
+            // chunk n-2 left this Y buffer (both long done: waited while the
+            // state warps still convert S), the bf16 state of chunk n written.
+            if (!warp_wait(&bar[B_FULLA + s], (n >> 1) & 1, abort_flag)) break;
+            if (n >= 2 && !warp_wait(&bar[B_OREAD + s], ((n - 2) >> 1) & 1, abort_flag)) break;
+            if (leader) EFLA_TR(22, n);
+            if (!warp_wait(&bar[B_SBFULL], n & 1, abort_flag)) break;
+            tc_fence_after();
+            if (leader) {
+                EFLA_TR(20, n);
+                const uint64_t dA = sdesc_sw128(sa + SL_Q0 * SLOT, 16, 1024);
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(yu, dA + (((kk >> 2) * BOXSTRIDE + (kk & 3) * 32) >> 4),
-                                 dSB + ((part * 2 * SLOT + kk * 2048) >> 4), ID_N64, 1);
+                        mma_bf16(ty, dA + (((kk >> 2) * 2 * SLOT + (kk & 3) * 32) >> 4),
+                                 dSB + ((part * 2 * SLOT + kk * 2048) >> 4), ID_Y, part | kk);
                 mma_commit(&bar[B_DFULL]);
-            };
-            auto issue_SO = [&](int n) {  // S += K^T (D_hi + D_lo);  Y += M_hi D_hi + M_hi D_lo + M_lo D_hi
-                const uint32_t yu = tmem + T_YU + 64 * (n & 1);
-                const uint64_t dKt = sdesc_sw128(stage_addr(n) + SL_K0 * SLOT, BOXSTRIDE, 1024);
-                const uint64_t dM = sdesc_sw128(sbase + OFF_M + (n & 1) * 2 * SLOT, 16, 1024);
+                mma_commit(&bar[B_EMPTYA + s]);
+                EFLA_TR(24, n);
+                if (n >= 1) issue_O(n - 1);
+            }
+            __syncwarp();
+            // S += K^T (D_hi + D_lo) after part B landed (K) and D was written
+            if (!warp_wait(&bar[B_FULLB + s], (n >> 1) & 1, abort_flag)) break;
+            if (!warp_wait(&bar[B_DELTA], n & 1, abort_flag)) break;
+            tc_fence_after();
+            if (leader) {
+                EFLA_TR(21, n);
+                const uint64_t dKt = sdesc_sw128(sa + SL_K0 * SLOT, SLOT, 1024);
+                const uint64_t dD = dDB + ((s * 2 * SLOT) >> 4);
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + T_S, dKt + ((kk * 2048) >> 4), dDB + ((part * SLOT + kk * 2048) >> 4), ID_S, 1);
-                mma_commit(&bar[B_SFULL]);  // the state chain waits only for S
-#pragma unroll
-                for (int part = 0; part < 3; ++part) {
-                    const uint32_t moff = (part == 2) ? SLOT : 0, doff = (part == 1) ? SLOT : 0;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(yu, dM + ((moff + kk * 32) >> 4), dDB + ((doff + kk * 2048) >> 4), ID_N64, 1);
-                }
-                mma_commit(&bar[B_OFULL + (n & 1)]);
-                mma_commit(&bar[B_EMPTY + (n & 1)]);
-            };
-            // Event-driven issue: each product goes out as soon as its inputs are
-            // ready, the serial D / SO chain first, so Y(n+1) and G(n+2) fill the
-            // gaps while the state warps read TMEM.  Ordering rules:
-            //   D(n)  after -W/M of chunk n (a2) and the bf16 state (sb);
-            //   SO(n) after the bf16 D (delta);
-            //   Y(m)  after X(m), after O(m-2) left the Y buffer (oread[m%2]) and
-            //         after D(m-2) was issued: D(m-2) waits for the -W readout
-            //         of chunk m-2, the last reader of X K buffer m%2;
-            //   G(m)  after its TMA stage landed, G(m-1) was read (gempty) and
-            //         SO(m-2) was issued (so the commit that signals G(m)
-            //         also covers every earlier reader of the buffers that
-            //         chunk m's prep overwrites).
-            int nD = 0, nS = 0, nY = 0, nG = 0;
-            long long idle_since = clock64();
-            while (nS < nc) {
-                bool did = false;
-                if (nD < nc && nD == nS && nD < nY && mbar_test(&bar[B_A2FULL + (nD & 1)], (nD >> 1) & 1) &&
-                    mbar_test(&bar[B_SBFULL], nD & 1)) {
-                    tc_fence_after();
-                    EFLA_TR(20, nD); issue_D(nD++);
-                    did = true;
-                }
-                if (nS < nD && mbar_test(&bar[B_DELTA], nS & 1)) {
-                    tc_fence_after();
-                    EFLA_TR(21, nS); issue_SO(nS++);
-                    did = true;
-                }
-                if (nY < nc && nY < nG && nY <= nD + 1 && mbar_test(&bar[B_XFULL], nY & 1) &&
-                    (nY < 2 || mbar_test(&bar[B_OREAD + (nY & 1)], ((nY - 2) >> 1) & 1))) {
-                    tc_fence_after();
-                    EFLA_TR(22, nY); issue_Y(nY++);
-                    did = true;
-                }
-                if (nG < nc && nG <= nS + 1 && nG <= nY + 1 && mbar_test(&bar[B_FULL + (nG & 1)], (nG >> 1) & 1) &&
-                    (nG == 0 || mbar_test(&bar[B_GEMPTY], (nG - 1) & 1))) {
-                    tc_fence_after();
-                    EFLA_TR(23, nG); issue_G(nG++);
-                    did = true;
-                }
-                if (did) {
-                    idle_since = clock64();
-                } else if (*abort_flag) {
-                    break;
-                } else if (clock64() - idle_since > kWaitCycles) {
-                    *abort_flag = 1;
-                    raise_error(kErrTimeout);
-                    break;
-                }
+                        mma_bf16(tmem + T_S, dKt + ((kk * 2048) >> 4), dD + ((part * SLOT + kk * 2048) >> 4), ID_S, 1);
+                mma_commit(&bar[B_SFULL]);
+                EFLA_TR(25, n);
             }
-            // drain: wait (bounded, even after an abort) until every MMA issued has completed
-            mma_commit(&bar[B_DRAIN]);
-            int never = 0;
-            mbar_wait(&bar[B_DRAIN], 0, &never);
+            __syncwarp();
         }
+        if (n == nc && leader) issue_O(nc - 1);
+        __syncwarp();
+        // drain: wait (bounded, even after an abort) until every MMA issued has completed
+        if (leader) mma_commit(&bar[B_DRAIN]);
+        __syncwarp();
+        int never = 0;
+        mbar_wait(&bar[B_DRAIN], 0, &never);
     } else {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+        // Whole warp in the loop; lane 0 issues the copies.
+        const bool leader = lane == 0;
+        if (leader) {
             tma_prefetch(&tm_q);
             tma_prefetch(&tm_k);
-            tma_prefetch(&tm_v);
-            int last[2] = {-1, -1};
-            for (int n = 0; n < nc; ++n) {
-                const int s = n & 1;
-                if (n >= 2 && !mbar_wait(&bar[B_EMPTY + s], ((n >> 1) - 1) & 1, abort_flag)) break;
-                if (*abort_flag) break;
-                unsigned char *st = sm + s * STAGE;
-                uint64_t *fb = &bar[B_FULL + s];
-                mbar_expect_tx(fb, 5 * SLOT);
-                const int y = n * C, z = (int)bh;
-                tma_load_3d(st + SL_K0 * SLOT, &tm_k, fb, 0, y, z);
-                tma_load_3d(st + SL_K0 * SLOT + BOXSTRIDE, &tm_k, fb, 64, y, z);
+        }
+        const unsigned char *img = ws + (size_t)bh * nc * PREP_BYTES;
+        int lastA[2] = {-1, -1}, lastB[2] = {-1, -1};  // last chunk loaded per stage and part
+        for (int n = 0; n < nc; ++n) {
+            const int s = n & 1;
+            unsigned char *st = sm + s * STAGE;
+            const int y = n * C, z = (int)bh;
+            const unsigned char *src = img + (size_t)n * PREP_BYTES;
+            // part A: Q and -W, once Y of chunk n-2 no longer reads them
+            if (n >= 2 && !warp_wait(&bar[B_EMPTYA + s], ((n >> 1) - 1) & 1, abort_flag)) break;
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            if (leader) {
+                uint64_t *fb = &bar[B_FULLA + s];
+                mbar_expect_tx(fb, TX_A);
                 tma_load_3d(st + SL_Q0 * SLOT, &tm_q, fb, 0, y, z);
-                tma_load_3d(st + SL_Q0 * SLOT + BOXSTRIDE, &tm_q, fb, 64, y, z);
-                tma_load_3d(st + SL_V * SLOT, &tm_v, fb, j0, y, z);
-                last[s] = n;
+                tma_load_3d(st + (SL_Q0 + 2) * SLOT, &tm_q, fb, 64, y, z);
+                bulk_load(st + SL_W0 * SLOT, src + IMG_W, SLOT, fb);
+                bulk_load(st + (SL_W0 + 2) * SLOT, src + IMG_W + SLOT, SLOT, fb);
+                EFLA_TR(27, n);
             }
-            // drain: every copy this thread started has landed before the CTA exits
-            int never = 0;
-            for (int s = 0; s < 2; ++s)
-                if (last[s] >= 0) mbar_wait(&bar[B_FULL + s], (last[s] >> 1) & 1, &never);
+            __syncwarp();
+            lastA[s] = n;
+            // part B: K, M and U, once chunk n-2 is finished with them
+            if (n >= 2 && !warp_wait(&bar[B_EMPTYB + s], ((n >> 1) - 1) & 1, abort_flag)) break;
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            if (leader) {
+                uint64_t *fb = &bar[B_FULLB + s];
+                mbar_expect_tx(fb, TX_B);
+                tma_load_3d(st + SL_K0 * SLOT, &tm_k, fb, 0, y, z);
+                tma_load_3d(st + (SL_K0 + 1) * SLOT, &tm_k, fb, 64, y, z);
+                bulk_load(st + SL_M * SLOT, src + IMG_M, SLOT, fb);
+                bulk_load(st + SL_U * SLOT, src + IMG_U + half * UHALF, UHALF, fb);
+            }
+            __syncwarp();
+            lastB[s] = n;
+        }
+        // drain: every copy this warp started has landed before the CTA exits
+        // (a load is issued only after the previous one of its stage and part
+        // was consumed, so the last one issued is the only one that can be pending)
+        int never = 0;
+        for (int s = 0; s < 2; ++s) {
+            if (lastA[s] >= 0) mbar_wait(&bar[B_FULLA + s], (lastA[s] >> 1) & 1, &never);
+            if (lastB[s] >= 0) mbar_wait(&bar[B_FULLB + s], (lastB[s] >> 1) & 1, &never);
         }
     }
+    if (threadIdx.x == 0) bulk_wait0();  // the O stores this thread issued are complete
     __syncwarp();
     tc_fence_before();
     __syncthreads();
@@ -692,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// ---------------------------------------------------------------- T' kernel
+// ---------------------------------------------------------------- prep kernel
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -701,85 +643,157 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-constexpr int KLD = DK + 8;  // padded bf16 row stride of K: conflict-free mma.sync fragment loads
-struct TPrepSmem {
-    union {  // K is dead once K K^T is formed; T reuses its space (6 CTAs per SM instead of 4)
-        __nv_bfloat16 K[C][KLD];
+// B fragments of two adjacent 8-column tiles of a 16 x 16 block of a
+// row-major bf16 matrix ([k][n]): ldmatrix .x4 .trans hands thread (g, t)
+// the pairs (k = 2t, 2t+1 | +8; n = g) of each tile.
+__device__ __forceinline__ void ldsm_x4t(const void *p, uint32_t (&b0)[2], uint32_t (&b1)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(b0[0]), "=r"(b0[1]), "=r"(b1[0]), "=r"(b1[1])
+                 : "r"(ptx::smem_u32(p)));
+}
+// A fragment (16 x 16, row-major) of mma.sync m16n8k16 from four 8 x 8 matrices.
+__device__ __forceinline__ void ldsm_x4(const void *p, uint32_t (&a)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(ptx::smem_u32(p)));
+}
+// 16-byte global -> shared copy (cp.async), zero-filled when `valid` is false.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ptx::smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+constexpr int KLD = DK + 8;  // padded bf16 row stride: conflict-free fragment loads
+constexpr int kPrepThreads = 256;
+struct PrepSmem {
+    __nv_bfloat16 K[C][KLD];
+    __nv_bfloat16 V[C][KLD];
+    union {  // Q is dead once Q K^T is formed; T reuses its space
+        __nv_bfloat16 Q[C][KLD];
         float T[C * LDF];
     };
-    float A[C * LDF];
+    union {  // A is dead after the solve; T' as bf16 hi and lo (swizzled 64 x 64 boxes) reuses it
+        float A[C * LDF];
+        unsigned char TP[2][C * 128];
+    };
     float alpha[C];
 };
 
-// Per chunk (rows past L zero): alpha = gate(beta, ||k||^2); A = strictly-lower
-// (diag(alpha) K K^T) by mma.sync bf16 on the 20 lower 16 x 8 tiles;
-// T = (I + A)^{-1}; writes T' = T diag(alpha) as bf16 hi and lo boxes in the
-// 128-byte-swizzled image chunk_tc_kernel's descriptors read.  One CTA of 128
-// threads per (b, h, chunk); independent chunks, so latency hides across CTAs.
-__global__ void __launch_bounds__(128) chunk_T_kernel(const __nv_bfloat16 *__restrict__ k,
-                                                      const float *__restrict__ beta,
-                                                      unsigned char *__restrict__ xws, int L, int nc, int euler) {
-    extern __shared__ __align__(16) unsigned char tsm_raw[];
-    TPrepSmem &sm = *reinterpret_cast<TPrepSmem *>(tsm_raw);
+__device__ __forceinline__ uint32_t ld_pair(const __nv_bfloat16 *p) { return *reinterpret_cast<const uint32_t *>(p); }
+
+// One 16 x 8 tile of (X Y^T) over d_k = 128, X and Y rows in padded bf16 smem:
+// rows x0.., y0.. (mma.sync m16n8k16, fp32 accumulation).
+__device__ __forceinline__ void gram_tile(const __nv_bfloat16 (*X)[KLD], const __nv_bfloat16 (*Y)[KLD], int x0, int y0,
+                                          int g, int t, float (&acc)[4]) {
+#pragma unroll
+    for (int k0 = 0; k0 < DK; k0 += 16) {
+        const uint32_t a[4] = {ld_pair(&X[x0 + g][k0 + 2 * t]), ld_pair(&X[x0 + g + 8][k0 + 2 * t]),
+                               ld_pair(&X[x0 + g][k0 + 2 * t + 8]), ld_pair(&X[x0 + g + 8][k0 + 2 * t + 8])};
+        const uint32_t b[2] = {ld_pair(&Y[y0 + g][k0 + 2 * t]), ld_pair(&Y[y0 + g][k0 + 2 * t + 8])};
+        mma_bf16_16816(acc, a, b);
+    }
+}
+
+// Byte offset of element (r, c) in a 64-column bf16 box with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw128_elem(int r, int c) {
+    return (uint32_t)r * 128u + ((((uint32_t)c >> 3) ^ ((uint32_t)r & 7u)) << 4) + ((uint32_t)c & 7u) * 2u;
+}
+
+// Row tile i and column tile j (16 x 8 tiles of a 64 x 64 matrix) of tile
+// number idx: 0..19 are the tiles on or below the diagonal 16 x 16 blocks
+// (row by row), 20..31 the tiles above them.
+__device__ __forceinline__ void tile_ij(int idx, int &i, int &j) {
+    if (idx < 20) {
+        i = idx < 2 ? 0 : idx < 6 ? 1 : idx < 12 ? 2 : 3;
+        j = idx - i * (i + 1);
+    } else {
+        const int u = idx - 20;
+        i = u < 6 ? 0 : u < 10 ? 1 : 2;
+        j = i == 0 ? 2 + u : i == 1 ? u - 2 : u - 4;
+    }
+}
+
+// Everything about one chunk that does not depend on the state, written as
+// the workspace image chunk_tc_kernel reads (rows past L are zero):
+//   alpha = gate(beta, ||k||^2),  A = strictly-lower(diag(alpha) K K^T),
+//   T = (I + A)^{-1},  T' = T diag(alpha),
+//   -W = -T' K  (bf16),  M = lower-incl-diag(Q K^T)  (bf16),
+//   U = T' V  (fp32).
+// Products run on mma.sync with fp32 accumulation: bf16 q/k/v operands, T' as
+// a bf16 hi + lo pair, TF32 in the block rows of T.  One 256-thread CTA per
+// (b, h, chunk): independent chunks, so their latency overlaps across CTAs.
+__global__ void __launch_bounds__(kPrepThreads) chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                                     const __nv_bfloat16 *__restrict__ k,
+                                                                     const __nv_bfloat16 *__restrict__ v,
+                                                                     const float *__restrict__ beta,
+                                                                     unsigned char *__restrict__ ws, int L, int nc,
+                                                                     int euler) {
+    extern __shared__ __align__(16) unsigned char psm_raw[];
+    PrepSmem &sm = *reinterpret_cast<PrepSmem *>(psm_raw);
     const int p = threadIdx.x, w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
     const long gidx = blockIdx.x;
     const int chunk = (int)(gidx % nc);
     const long bh = gidx / nc;
     const int t0 = chunk * C, n = min(C, L - t0);
-    const __nv_bfloat16 *kc = k + ((size_t)bh * L + t0) * DK;
-    for (int e = p; e < C * (DK / 8); e += 128) {
-        const int r = e / (DK / 8), c8 = (e % (DK / 8)) * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < n) v = __ldg(reinterpret_cast<const uint4 *>(kc + (size_t)r * DK + c8));
-        *reinterpret_cast<uint4 *>(&sm.K[r][c8]) = v;
+    const size_t row0 = (size_t)bh * L + t0;
+#pragma unroll
+    for (int it = 0; it < C * (DK / 8) / kPrepThreads; ++it) {
+        const int e = p + kPrepThreads * it, r = e >> 4, c8 = (e & 15) * 8;
+        const bool ok = r < n;
+        const size_t go = (row0 + (ok ? r : 0)) * DK + c8;
+        cp_async16(&sm.K[r][c8], k + go, ok);
+        cp_async16(&sm.Q[r][c8], q + go, ok);
+        cp_async16(&sm.V[r][c8], v + go, ok);
     }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     __syncthreads();
-    {   // gate: two lanes per key row
-        const int r = p >> 1, h = p & 1;
+    {   // gate: four lanes per key row
+        const int r = p >> 2, h = p & 3;
         float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
             float f[8];
-            unpack8(*reinterpret_cast<const uint4 *>(&sm.K[r][64 * h + 8 * j]), f);
+            unpack8(*reinterpret_cast<const uint4 *>(&sm.K[r][32 * h + 8 * j]), f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc8[e] = fmaf(f[e], f[e], acc8[e]);
         }
         float ss = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        if (h == 0) sm.alpha[r] = (r < n) ? gate_alpha(beta[bh * (long)L + t0 + r], ss, euler != 0) : 0.f;
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        if (h == 0) sm.alpha[r] = (r < n) ? gate_alpha(beta[row0 + r], ss, euler != 0) : 0.f;
     }
     __syncthreads();
+    unsigned char *out = ws + (size_t)gidx * PREP_BYTES;
     const Split64 Af{sm.A, sm.A + 32 * LDF}, Tf{sm.T, sm.T + 32 * LDF};
-    // the 20 tiles (row tile i of 16, column tile j of 8) on or below the diagonal blocks
-    for (int tile = w; tile < 20; tile += 4) {
-        int i = 0, j = tile;
-        while (j >= 2 * i + 2) {
-            j -= 2 * i + 2;
-            ++i;
-        }
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k0 = 0; k0 < DK; k0 += 16) {
-            const uint32_t a[4] = {*reinterpret_cast<const uint32_t *>(&sm.K[16 * i + g][k0 + 2 * t]),
-                                   *reinterpret_cast<const uint32_t *>(&sm.K[16 * i + g + 8][k0 + 2 * t]),
-                                   *reinterpret_cast<const uint32_t *>(&sm.K[16 * i + g][k0 + 2 * t + 8]),
-                                   *reinterpret_cast<const uint32_t *>(&sm.K[16 * i + g + 8][k0 + 2 * t + 8])};
-            const uint32_t b[2] = {*reinterpret_cast<const uint32_t *>(&sm.K[8 * j + g][k0 + 2 * t]),
-                                   *reinterpret_cast<const uint32_t *>(&sm.K[8 * j + g][k0 + 2 * t + 8])};
-            mma_bf16_16816(acc, a, b);
-        }
+    // A (from K K^T) and M (from Q K^T) on the tiles on or below the diagonal
+    // blocks; M's other tiles are zero.
+#pragma unroll 1
+    for (int idx = w; idx < 32; idx += kPrepThreads / 32) {
+        int i, j;
+        tile_ij(idx, i, j);
         const int r0 = 16 * i + g, r1 = r0 + 8, c0 = 8 * j + 2 * t;
-        *Af.at(r0, c0) = (c0 < r0) ? sm.alpha[r0] * acc[0] : 0.f;
-        *Af.at(r0, c0 + 1) = (c0 + 1 < r0) ? sm.alpha[r0] * acc[1] : 0.f;
-        *Af.at(r1, c0) = (c0 < r1) ? sm.alpha[r1] * acc[2] : 0.f;
-        *Af.at(r1, c0 + 1) = (c0 + 1 < r1) ? sm.alpha[r1] * acc[3] : 0.f;
+        float qk[4] = {0.f, 0.f, 0.f, 0.f};
+        if (idx < 20) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            gram_tile(sm.K, sm.K, 16 * i, 8 * j, g, t, acc);
+            *Af.at(r0, c0) = (c0 < r0) ? sm.alpha[r0] * acc[0] : 0.f;
+            *Af.at(r0, c0 + 1) = (c0 + 1 < r0) ? sm.alpha[r0] * acc[1] : 0.f;
+            *Af.at(r1, c0) = (c0 < r1) ? sm.alpha[r1] * acc[2] : 0.f;
+            *Af.at(r1, c0 + 1) = (c0 + 1 < r1) ? sm.alpha[r1] * acc[3] : 0.f;
+            gram_tile(sm.Q, sm.K, 16 * i, 8 * j, g, t, qk);
+        }
+        *reinterpret_cast<uint32_t *>(out + IMG_M + sw128_elem(r0, c0)) =
+            ptx::pack_bf16((c0 <= r0) ? qk[0] : 0.f, (c0 + 1 <= r0) ? qk[1] : 0.f);
+        *reinterpret_cast<uint32_t *>(out + IMG_M + sw128_elem(r1, c0)) =
+            ptx::pack_bf16((c0 <= r1) ? qk[2] : 0.f, (c0 + 1 <= r1) ? qk[3] : 0.f);
     }
-    __syncthreads();
-    invert_unit_lower(p, Af, Tf);
-    unsigned char *dst = xws + (size_t)gidx * XBYTES;
+    __syncthreads();  // Q is dead from here; its space becomes T
+    invert_unit_lower<kPrepThreads>(p, Af, Tf);
+    // T' = T diag(alpha) (lower triangle) as swizzled bf16 hi and lo boxes in A's space
 #pragma unroll
-    for (int ii = 0; ii < 4; ++ii) {
-        const int e = p + 128 * ii, r = e >> 3, jj = e & 7;
+    for (int it = 0; it < 2; ++it) {
+        const int e = p + kPrepThreads * it, r = e >> 3, jj = e & 7;
         const float4 ta = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * jj));
         const float4 tb = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * jj + 4));
         const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
@@ -787,12 +801,57 @@ __global__ void __launch_bounds__(128) chunk_T_kernel(const __nv_bfloat16 *__res
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int c = 8 * jj + 2 * u;
-            const float x0 = (c <= r) ? tv[2 * u] * sm.alpha[c] : 0.f;
-            const float x1 = (c + 1 <= r) ? tv[2 * u + 1] * sm.alpha[c + 1] : 0.f;
-            split2(x0, x1, h4[u], l4[u]);
+            split2((c <= r) ? tv[2 * u] * sm.alpha[c] : 0.f, (c + 1 <= r) ? tv[2 * u + 1] * sm.alpha[c + 1] : 0.f,
+                   h4[u], l4[u]);
         }
-        *reinterpret_cast<uint4 *>(dst + ptx::sw128_chunk(r, jj)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-        *reinterpret_cast<uint4 *>(dst + SLOT + ptx::sw128_chunk(r, jj)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+        *reinterpret_cast<uint4 *>(sm.TP[0] + ptx::sw128_chunk(r, jj)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+        *reinterpret_cast<uint4 *>(sm.TP[1] + ptx::sw128_chunk(r, jj)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
+    }
+    __syncthreads();
+    // -W = -T' K and U = T' V: warp w owns the 8-column tiles 2w and 2w+1 of
+    // both, for all four 16-row tiles; T' is lower triangular, so row tile i
+    // needs k < 16 (i + 1).  ldmatrix lane l addresses row (l & 7) + 8 ((l >> 3) & 1)
+    // of the 16-row block and 8-column group (l >> 4).
+    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lgrp = lane >> 4;
+#pragma unroll 1
+    for (int i = 0; i < 4; ++i) {
+        float aw[2][4], au[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) aw[u][e] = au[u][e] = 0.f;
+        const int ar = 16 * i + lrow;
+#pragma unroll 1
+        for (int k0 = 0; k0 < 16 * (i + 1); k0 += 16) {
+            uint32_t ah[4], al[4], bk0[2], bk1[2], bv0[2], bv1[2];
+            const uint32_t aoff = ptx::sw128_chunk(ar, (k0 >> 3) + lgrp);
+            ldsm_x4(sm.TP[0] + aoff, ah);
+            ldsm_x4(sm.TP[1] + aoff, al);
+            ldsm_x4t(&sm.K[k0 + lrow][8 * (2 * w + lgrp)], bk0, bk1);
+            ldsm_x4t(&sm.V[k0 + lrow][8 * (2 * w + lgrp)], bv0, bv1);
+            mma_bf16_16816(aw[0], ah, bk0);
+            mma_bf16_16816(aw[1], ah, bk1);
+            mma_bf16_16816(au[0], ah, bv0);
+            mma_bf16_16816(au[1], ah, bv1);
+            mma_bf16_16816(aw[0], al, bk0);
+            mma_bf16_16816(aw[1], al, bk1);
+            mma_bf16_16816(au[0], al, bv0);
+            mma_bf16_16816(au[1], al, bv1);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int c = 8 * (2 * w + u) + 2 * t;  // d column, 0..127
+            const int box = c >> 6, cc = c & 63;
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int r = 16 * i + g + 8 * hr;
+                *reinterpret_cast<uint32_t *>(out + IMG_W + box * SLOT + sw128_elem(r, cc)) =
+                    ptx::pack_bf16(-aw[u][2 * hr], -aw[u][2 * hr + 1]);
+                const uint32_t uo =
+                    IMG_U + box * UHALF + r * 256 + ((((uint32_t)cc >> 2) ^ ((uint32_t)r & 15u)) << 4) + (cc & 3) * 4;
+                *reinterpret_cast<float2 *>(out + uo) = make_float2(au[u][2 * hr], au[u][2 * hr + 1]);
+            }
+        }
     }
 }
 
@@ -814,39 +873,48 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D view [bh][L][128] of a bf16 [B][H][L][128] tensor, 64 x 64 boxes,
-// 128-byte swizzle; rows past L read as zero.
-inline bool make_map(CUtensorMap *m, const void *base, long bh, int L) {
+// 3-D view [bh][L][128] of a [B][H][L][128] tensor, boxes of bx columns x 64
+// rows with the 128-byte swizzle; rows past L read as zero (loads) and are
+// not written (stores).
+inline bool make_map(CUtensorMap *m, const void *base, long bh, int L, CUtensorMapDataType dt, int esize,
+                     unsigned bx) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)L, (cuuint64_t)bh};
-    const cuuint64_t strides[2] = {(cuuint64_t)DK * 2, (cuuint64_t)L * DK * 2};
-    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint64_t strides[2] = {(cuuint64_t)DK * esize, (cuuint64_t)L * DK * esize};
+    const cuuint32_t box[3] = {bx, 64, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+inline bool make_map_bf16_sw128(CUtensorMap *m, const void *base, long bh, int L) {
+    return make_map(m, base, bh, L, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64);
 }
 
-// Scratch of the tensor-core path: one T' image (hi + lo boxes) per chunk.
-inline size_t workspace_bytes(long bh, int L) { return (size_t)bh * ((L + C - 1) / C) * XBYTES; }
+// Scratch of the tensor-core path: one -W / M / U image per chunk.
+inline size_t workspace_bytes(long bh, int L) { return (size_t)bh * ((L + C - 1) / C) * PREP_BYTES; }
 
 template <typename Tout>
 inline efla_status_t launch(const void *q, const void *k, const void *v, const float *beta, const float *S0,
                             void *o, float *SL, long bh, int L, bool euler, void *ws, cudaStream_t st) {
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, bh, L) || !make_map(&mk, k, bh, L) || !make_map(&mv, v, bh, L)) return EFLA_ERR_CUDA;
-    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES) || !ensure_smem<chunk_T_kernel>(sizeof(TPrepSmem)))
+    CUtensorMap mq, mk, mo;
+    const bool of32 = sizeof(Tout) == 4;
+    if (!make_map_bf16_sw128(&mq, q, bh, L) || !make_map_bf16_sw128(&mk, k, bh, L) ||
+        !make_map(&mo, o, bh, L, of32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  (int)sizeof(Tout), of32 ? 32u : 64u))
+        return EFLA_ERR_CUDA;
+    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES) || !ensure_smem<chunk_prep_tc_kernel>(sizeof(PrepSmem)))
         return EFLA_ERR_CUDA;
     const long grid = bh * NSPLIT;
     const int nc = (L + C - 1) / C;
     if (grid > 0x7fffffffL || bh * nc > 0x7fffffffL) return EFLA_ERR_SHAPE;
-    unsigned char *xws = static_cast<unsigned char *>(ws);
-    chunk_T_kernel<<<(unsigned)(bh * nc), 128, sizeof(TPrepSmem), st>>>(static_cast<const __nv_bfloat16 *>(k), beta,
-                                                                        xws, L, nc, euler ? 1 : 0);
+    unsigned char *img = static_cast<unsigned char *>(ws);
+    chunk_prep_tc_kernel<<<(unsigned)(bh * nc), kPrepThreads, sizeof(PrepSmem), st>>>(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), beta, img, L, nc, euler ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
-    chunk_tc_kernel<Tout><<<(unsigned)grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mv, xws, S0, static_cast<Tout *>(o),
-                                                                         SL, L, nc);
+    chunk_tc_kernel<Tout><<<(unsigned)grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mo, img, S0, SL, L, nc);
     return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
 }
 
