@@ -164,21 +164,25 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
     }
 }
 
-// A 64 x 64 fp32 matrix stored as two 32-row halves of 256-byte rows.  The
-// 16-byte slots of row r are XOR-permuted by (r & 15), so row-per-thread
-// float4 stores and same-column loads across rows hit distinct banks.
-struct Split64 {
-    float *lo, *hi;
-    __device__ __forceinline__ float *row(int r) const { return (r < 32 ? lo : hi) + (r & 31) * LDF; }
+// A 64 x 64 fp32 matrix of 256-byte rows whose 16-byte slots are XOR-permuted
+// by (r & 15), so row-per-thread float4 stores and same-column loads across
+// rows hit distinct banks.
+struct Sw64 {
+    float *p;
     // element (r, c); for c % 4 == 0 this is the start of a contiguous float4
     __device__ __forceinline__ float *at(int r, int c) const {
-        return row(r) + ((((c >> 2) ^ (r & 15)) << 2) | (c & 3));
+        return p + r * LDF + ((((c >> 2) ^ (r & 15)) << 2) | (c & 3));
     }
 };
 
+// Diagonal 16 x 16 blocks of A, laid out for the forward substitution: block
+// b, column m, row parity h, then the 8 rows 2s + h (s = 0..7) contiguous.
+__device__ __forceinline__ int diag_index(int b, int m, int h, int s) { return ((b * 16 + m) * 2 + h) * 8 + s; }
+
 // T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A.  First the
 // four 16 x 16 diagonal blocks by right-looking forward substitution (warps
-// 0-3, one block each, one column per lane pair, fp32); then block rows
+// 0-3, one block each, one column per lane pair, fp32, A's diagonal blocks
+// read from their own copy Ad); then block rows
 // I = 1..3:
 //     R = A_{I,<I} T_{<I,<I},   T_{I,<I} = -T_II R,
 // as 16 x 8 tiles on mma.sync (TF32 operands, fp32 accumulation).  TF32
@@ -187,7 +191,8 @@ struct Split64 {
 // oracle with fp32 or TF32 block products.  NT threads (a multiple of 128)
 // call it together; it ends with all of them synchronised on barrier 1.
 template <int NT>
-__device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af, const Split64 Tf) {
+__device__ __forceinline__ void invert_unit_lower(const int p, const float *__restrict__ Ad, const Sw64 Af,
+                                                  const Sw64 Tf) {
     if (p < 128) {
         const int w = p >> 5, l = p & 31, c = l & 15, h = l >> 4, base = 16 * w;
         float acc[8];
@@ -196,8 +201,11 @@ __device__ __forceinline__ void invert_unit_lower(const int p, const Split64 Af,
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
             const float x = __shfl_sync(0xffffffffu, acc[m >> 1], ((m & 1) << 4) | c);
+            const float4 a0 = *reinterpret_cast<const float4 *>(Ad + diag_index(w, m, h, 0));
+            const float4 a1 = *reinterpret_cast<const float4 *>(Ad + diag_index(w, m, h, 4));
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-            for (int s = 0; s < 8; ++s) acc[s] = fmaf(-*Af.at(base + 2 * s + h, base + m), x, acc[s]);
+            for (int s = 0; s < 8; ++s) acc[s] = fmaf(-a[s], x, acc[s]);
         }
 #pragma unroll
         for (int s = 0; s < 8; ++s) *Tf.at(base + 2 * s + h, base + c) = acc[s];
@@ -677,21 +685,33 @@ struct PrepSmem {
         float A[C * LDF];
         unsigned char TP[2][C * 128];
     };
+    float Ad[4 * 16 * 16];  // diagonal 16 x 16 blocks of A for the forward substitution (diag_index)
     float alpha[C];
 };
 
-__device__ __forceinline__ uint32_t ld_pair(const __nv_bfloat16 *p) { return *reinterpret_cast<const uint32_t *>(p); }
+// ldmatrix .x2: B fragments (col-major, 16 x 8) of one 8-column tile.
+__device__ __forceinline__ void ldsm_x2(const void *p, uint32_t (&b)[2]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(b[0]), "=r"(b[1])
+                 : "r"(ptx::smem_u32(p)));
+}
 
-// One 16 x 8 tile of (X Y^T) over d_k = 128, X and Y rows in padded bf16 smem:
-// rows x0.., y0.. (mma.sync m16n8k16, fp32 accumulation).
-__device__ __forceinline__ void gram_tile(const __nv_bfloat16 (*X)[KLD], const __nv_bfloat16 (*Y)[KLD], int x0, int y0,
-                                          int g, int t, float (&acc)[4]) {
+// One 16 x 8 tile of K K^T and of Q K^T over d_k = 128 (rows x0.. of K and
+// Q, columns y0.. = rows y0.. of K), sharing the B fragments; fragments come
+// from padded bf16 rows through ldmatrix.  lrow / lgrp: this lane's ldmatrix
+// row within a 16-row block and 8-column group.
+__device__ __forceinline__ void gram2_tile(const __nv_bfloat16 (*K)[KLD], const __nv_bfloat16 (*Q)[KLD], int x0,
+                                           int y0, int lane, float (&kk)[4], float (&qk)[4]) {
+    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lgrp = lane >> 4;
+    const int brow = y0 + (lane & 7), bgrp = (lane >> 3) & 1;
 #pragma unroll
     for (int k0 = 0; k0 < DK; k0 += 16) {
-        const uint32_t a[4] = {ld_pair(&X[x0 + g][k0 + 2 * t]), ld_pair(&X[x0 + g + 8][k0 + 2 * t]),
-                               ld_pair(&X[x0 + g][k0 + 2 * t + 8]), ld_pair(&X[x0 + g + 8][k0 + 2 * t + 8])};
-        const uint32_t b[2] = {ld_pair(&Y[y0 + g][k0 + 2 * t]), ld_pair(&Y[y0 + g][k0 + 2 * t + 8])};
-        mma_bf16_16816(acc, a, b);
+        uint32_t ak[4], aq[4], b[2];
+        ldsm_x4(&K[x0 + lrow][k0 + 8 * lgrp], ak);
+        ldsm_x4(&Q[x0 + lrow][k0 + 8 * lgrp], aq);
+        ldsm_x2(&K[brow][k0 + 8 * bgrp], b);
+        mma_bf16_16816(kk, ak, b);
+        mma_bf16_16816(qk, aq, b);
     }
 }
 
@@ -765,9 +785,10 @@ __global__ void __launch_bounds__(kPrepThreads) chunk_prep_tc_kernel(const __nv_
     }
     __syncthreads();
     unsigned char *out = ws + (size_t)gidx * PREP_BYTES;
-    const Split64 Af{sm.A, sm.A + 32 * LDF}, Tf{sm.T, sm.T + 32 * LDF};
+    const Sw64 Af{sm.A}, Tf{sm.T};
     // A (from K K^T) and M (from Q K^T) on the tiles on or below the diagonal
-    // blocks; M's other tiles are zero.
+    // blocks; M's other tiles are zero.  A's diagonal blocks go to Ad, the
+    // blocks left of them to Af.
 #pragma unroll 1
     for (int idx = w; idx < 32; idx += kPrepThreads / 32) {
         int i, j;
@@ -775,13 +796,20 @@ __global__ void __launch_bounds__(kPrepThreads) chunk_prep_tc_kernel(const __nv_
         const int r0 = 16 * i + g, r1 = r0 + 8, c0 = 8 * j + 2 * t;
         float qk[4] = {0.f, 0.f, 0.f, 0.f};
         if (idx < 20) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            gram_tile(sm.K, sm.K, 16 * i, 8 * j, g, t, acc);
-            *Af.at(r0, c0) = (c0 < r0) ? sm.alpha[r0] * acc[0] : 0.f;
-            *Af.at(r0, c0 + 1) = (c0 + 1 < r0) ? sm.alpha[r0] * acc[1] : 0.f;
-            *Af.at(r1, c0) = (c0 < r1) ? sm.alpha[r1] * acc[2] : 0.f;
-            *Af.at(r1, c0 + 1) = (c0 + 1 < r1) ? sm.alpha[r1] * acc[3] : 0.f;
-            gram_tile(sm.Q, sm.K, 16 * i, 8 * j, g, t, qk);
+            float kk[4] = {0.f, 0.f, 0.f, 0.f};
+            gram2_tile(sm.K, sm.Q, 16 * i, 8 * j, lane, kk, qk);
+            const float a00 = (c0 < r0) ? sm.alpha[r0] * kk[0] : 0.f, a01 = (c0 + 1 < r0) ? sm.alpha[r0] * kk[1] : 0.f;
+            const float a10 = (c0 < r1) ? sm.alpha[r1] * kk[2] : 0.f, a11 = (c0 + 1 < r1) ? sm.alpha[r1] * kk[3] : 0.f;
+            if ((j >> 1) == i) {  // diagonal block: column m = c - 16 i, row 2 s + h = r - 16 i
+                const int m = c0 - 16 * i, s0 = g >> 1, h = g & 1;
+                sm.Ad[diag_index(i, m, h, s0)] = a00;
+                sm.Ad[diag_index(i, m + 1, h, s0)] = a01;
+                sm.Ad[diag_index(i, m, h, s0 + 4)] = a10;
+                sm.Ad[diag_index(i, m + 1, h, s0 + 4)] = a11;
+            } else {
+                *reinterpret_cast<float2 *>(Af.at(r0, c0)) = make_float2(a00, a01);
+                *reinterpret_cast<float2 *>(Af.at(r1, c0)) = make_float2(a10, a11);
+            }
         }
         *reinterpret_cast<uint32_t *>(out + IMG_M + sw128_elem(r0, c0)) =
             ptx::pack_bf16((c0 <= r0) ? qk[0] : 0.f, (c0 + 1 <= r0) ? qk[1] : 0.f);
@@ -789,7 +817,7 @@ __global__ void __launch_bounds__(kPrepThreads) chunk_prep_tc_kernel(const __nv_
             ptx::pack_bf16((c0 <= r1) ? qk[2] : 0.f, (c0 + 1 <= r1) ? qk[3] : 0.f);
     }
     __syncthreads();  // Q is dead from here; its space becomes T
-    invert_unit_lower<kPrepThreads>(p, Af, Tf);
+    invert_unit_lower<kPrepThreads>(p, sm.Ad, Af, Tf);
     // T' = T diag(alpha) (lower triangle) as swizzled bf16 hi and lo boxes in A's space
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
