@@ -179,20 +179,23 @@ struct Sw64 {
 // b, column m, row parity h, then the 8 rows 2s + h (s = 0..7) contiguous.
 __device__ __forceinline__ int diag_index(int b, int m, int h, int s) { return ((b * 16 + m) * 2 + h) * 8 + s; }
 
-// T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A.  First the
-// four 16 x 16 diagonal blocks by right-looking forward substitution (warps
-// 0-3, one block each, one column per lane pair, fp32, A's diagonal blocks
-// read from their own copy Ad); then block rows
-// I = 1..3:
+// T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A, in place:
+// AT holds A's blocks left of the diagonal on entry and T's lower triangle
+// (diagonal blocks included) on return.  First the four 16 x 16 diagonal
+// blocks by right-looking forward substitution (warps 0-3, one block each,
+// one column per lane pair, fp32, A's diagonal blocks read from their own
+// copy Ad); then block rows I = 1..3:
 //     R = A_{I,<I} T_{<I,<I},   T_{I,<I} = -T_II R,
-// as 16 x 8 tiles on mma.sync (TF32 operands, fp32 accumulation).  TF32
-// here costs nothing measurable: T then feeds bf16 hi/lo operands, and an
-// emulation of the whole computation gave the same error against the
-// oracle with fp32 or TF32 block products.  NT threads (a multiple of 128)
-// call it together; it ends with all of them synchronised on barrier 1.
+// as 16 x 8 tiles on mma.sync (TF32 operands, fp32 accumulation), warp w
+// owning column tile w.  TF32 here costs nothing measurable: T then feeds
+// bf16 hi/lo operands, and an emulation of the whole computation gave the
+// same error against the oracle with fp32 or TF32 block products.  Every R
+// of a block row is formed (and parked in Ad, free by then) before any of
+// its T tiles overwrites the A tiles the others still read.  NT = 256
+// threads call it together; it ends with all of them synchronised.
 template <int NT>
-__device__ __forceinline__ void invert_unit_lower(const int p, const float *__restrict__ Ad, const Sw64 Af,
-                                                  const Sw64 Tf) {
+__device__ __forceinline__ void invert_unit_lower(const int p, float *__restrict__ Ad, const Sw64 AT) {
+    static_assert(NT / 32 >= 6, "one warp per column tile of the last block row");
     if (p < 128) {
         const int w = p >> 5, l = p & 31, c = l & 15, h = l >> 4, base = 16 * w;
         float acc[8];
@@ -208,55 +211,45 @@ __device__ __forceinline__ void invert_unit_lower(const int p, const float *__re
             for (int s = 0; s < 8; ++s) acc[s] = fmaf(-a[s], x, acc[s]);
         }
 #pragma unroll
-        for (int s = 0; s < 8; ++s) *Tf.at(base + 2 * s + h, base + c) = acc[s];
+        for (int s = 0; s < 8; ++s) *AT.at(base + 2 * s + h, base + c) = acc[s];
     }
     ptx::named_bar(1, NT);
-    // Block rows on the tensor cores through mma.sync m16n8k8 (TF32 inputs,
-    // fp32 accumulation): warp w owns the 8-column tiles jt = w, w + NT/32, ...
-    // of block row I, so R's tile and the T tile computed from it stay inside
-    // one warp.  R is parked in T's own slots between the two products.
+    if (p == 0) EFLA_TR(55, 1023);
     const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
+    float *park = Ad + w * 128;  // this warp's 16 x 8 R tile, row-major
 #pragma unroll 1
     for (int I = 1; I < 4; ++I) {
-        const int r0 = 16 * I;
-#pragma unroll 1
-        for (int jt = w; jt < 2 * I; jt += NT / 32) {
-            const int c0 = 8 * jt;
+        const int r0 = 16 * I, c0 = 8 * w;
+        const bool mine = w < 2 * I;
+        if (mine) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             // R tile = A[r0.., k] T[k, c0..] over k from the column's own block up to r0
 #pragma unroll 1
-            for (int k0 = 16 * (jt >> 1); k0 < r0; k0 += 8) {
-                const uint32_t a[4] = {f2tf32(*Af.at(r0 + g, k0 + t)), f2tf32(*Af.at(r0 + g + 8, k0 + t)),
-                                       f2tf32(*Af.at(r0 + g, k0 + t + 4)), f2tf32(*Af.at(r0 + g + 8, k0 + t + 4))};
-                const uint32_t bb[2] = {f2tf32(*Tf.at(k0 + t, c0 + g)), f2tf32(*Tf.at(k0 + t + 4, c0 + g))};
+            for (int k0 = 16 * (w >> 1); k0 < r0; k0 += 8) {
+                const uint32_t a[4] = {f2tf32(*AT.at(r0 + g, k0 + t)), f2tf32(*AT.at(r0 + g + 8, k0 + t)),
+                                       f2tf32(*AT.at(r0 + g, k0 + t + 4)), f2tf32(*AT.at(r0 + g + 8, k0 + t + 4))};
+                const uint32_t bb[2] = {f2tf32(*AT.at(k0 + t, c0 + g)), f2tf32(*AT.at(k0 + t + 4, c0 + g))};
                 mma_tf32(acc, a, bb);
             }
-            *Tf.at(r0 + g, c0 + 2 * t) = acc[0];
-            *Tf.at(r0 + g, c0 + 2 * t + 1) = acc[1];
-            *Tf.at(r0 + g + 8, c0 + 2 * t) = acc[2];
-            *Tf.at(r0 + g + 8, c0 + 2 * t + 1) = acc[3];
-            __syncwarp();
-            uint32_t rb[2][2];
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-                rb[kk][0] = f2tf32(*Tf.at(r0 + 8 * kk + t, c0 + g));
-                rb[kk][1] = f2tf32(*Tf.at(r0 + 8 * kk + t + 4, c0 + g));
-            }
-            __syncwarp();
+            *reinterpret_cast<float2 *>(park + g * 8 + 2 * t) = make_float2(acc[0], acc[1]);
+            *reinterpret_cast<float2 *>(park + (g + 8) * 8 + 2 * t) = make_float2(acc[2], acc[3]);
+        }
+        ptx::named_bar(1, NT);  // every R formed: block row I of A may now be overwritten
+        if (mine) {
             float out[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {  // T tile = -T_II R tile
                 const int k0 = r0 + 8 * kk;
-                const uint32_t a[4] = {f2tf32(*Tf.at(r0 + g, k0 + t)), f2tf32(*Tf.at(r0 + g + 8, k0 + t)),
-                                       f2tf32(*Tf.at(r0 + g, k0 + t + 4)), f2tf32(*Tf.at(r0 + g + 8, k0 + t + 4))};
-                mma_tf32(out, a, rb[kk]);
+                const uint32_t a[4] = {f2tf32(*AT.at(r0 + g, k0 + t)), f2tf32(*AT.at(r0 + g + 8, k0 + t)),
+                                       f2tf32(*AT.at(r0 + g, k0 + t + 4)), f2tf32(*AT.at(r0 + g + 8, k0 + t + 4))};
+                const uint32_t bb[2] = {f2tf32(park[(8 * kk + t) * 8 + g]), f2tf32(park[(8 * kk + t + 4) * 8 + g])};
+                mma_tf32(out, a, bb);
             }
-            *Tf.at(r0 + g, c0 + 2 * t) = -out[0];
-            *Tf.at(r0 + g, c0 + 2 * t + 1) = -out[1];
-            *Tf.at(r0 + g + 8, c0 + 2 * t) = -out[2];
-            *Tf.at(r0 + g + 8, c0 + 2 * t + 1) = -out[3];
+            *reinterpret_cast<float2 *>(AT.at(r0 + g, c0 + 2 * t)) = make_float2(-out[0], -out[1]);
+            *reinterpret_cast<float2 *>(AT.at(r0 + g + 8, c0 + 2 * t)) = make_float2(-out[2], -out[3]);
         }
         ptx::named_bar(1, NT);
+        if (p == 0) EFLA_TR(55 + I, 1023);
     }
 }
 
@@ -643,243 +636,254 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- prep kernel
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// B fragments of two adjacent 8-column tiles of a 16 x 16 block of a
-// row-major bf16 matrix ([k][n]): ldmatrix .x4 .trans hands thread (g, t)
-// the pairs (k = 2t, 2t+1 | +8; n = g) of each tile.
-__device__ __forceinline__ void ldsm_x4t(const void *p, uint32_t (&b0)[2], uint32_t (&b1)[2]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(b0[0]), "=r"(b0[1]), "=r"(b1[0]), "=r"(b1[1])
-                 : "r"(ptx::smem_u32(p)));
-}
-// A fragment (16 x 16, row-major) of mma.sync m16n8k16 from four 8 x 8 matrices.
-__device__ __forceinline__ void ldsm_x4(const void *p, uint32_t (&a)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
-                 : "r"(ptx::smem_u32(p)));
-}
-// 16-byte global -> shared copy (cp.async), zero-filled when `valid` is false.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(ptx::smem_u32(dst)), "l"(src),
-                 "r"(valid ? 16 : 0)
-                 : "memory");
-}
-
-constexpr int KLD = DK + 8;  // padded bf16 row stride: conflict-free fragment loads
 constexpr int kPrepThreads = 256;
-struct PrepSmem {
-    __nv_bfloat16 K[C][KLD];
-    __nv_bfloat16 V[C][KLD];
-    union {  // Q is dead once Q K^T is formed; T reuses its space
-        __nv_bfloat16 Q[C][KLD];
-        float T[C * LDF];
-    };
-    union {  // A is dead after the solve; T' as bf16 hi and lo (swizzled 64 x 64 boxes) reuses it
-        float A[C * LDF];
-        unsigned char TP[2][C * 128];
-    };
-    float Ad[4 * 16 * 16];  // diagonal 16 x 16 blocks of A for the forward substitution (diag_index)
-    float alpha[C];
-};
-
-// ldmatrix .x2: B fragments (col-major, 16 x 8) of one 8-column tile.
-__device__ __forceinline__ void ldsm_x2(const void *p, uint32_t (&b)[2]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-                 : "=r"(b[0]), "=r"(b[1])
-                 : "r"(ptx::smem_u32(p)));
-}
-
-// One 16 x 8 tile of K K^T and of Q K^T over d_k = 128 (rows x0.. of K and
-// Q, columns y0.. = rows y0.. of K), sharing the B fragments; fragments come
-// from padded bf16 rows through ldmatrix.  lrow / lgrp: this lane's ldmatrix
-// row within a 16-row block and 8-column group.
-__device__ __forceinline__ void gram2_tile(const __nv_bfloat16 (*K)[KLD], const __nv_bfloat16 (*Q)[KLD], int x0,
-                                           int y0, int lane, float (&kk)[4], float (&qk)[4]) {
-    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lgrp = lane >> 4;
-    const int brow = y0 + (lane & 7), bgrp = (lane >> 3) & 1;
-#pragma unroll
-    for (int k0 = 0; k0 < DK; k0 += 16) {
-        uint32_t ak[4], aq[4], b[2];
-        ldsm_x4(&K[x0 + lrow][k0 + 8 * lgrp], ak);
-        ldsm_x4(&Q[x0 + lrow][k0 + 8 * lgrp], aq);
-        ldsm_x2(&K[brow][k0 + 8 * bgrp], b);
-        mma_bf16_16816(kk, ak, b);
-        mma_bf16_16816(qk, aq, b);
-    }
-}
+// Shared memory of one prep CTA (base aligned to 1024 B):
+//   [0, 32K)   K0 Q0 K1 Q1 (64 x 64 bf16 boxes, 128-byte swizzle): [K; Q] is
+//              the 128-row A operand of [K; Q] K^T per d_k half, K also its B;
+//              V0 and V1 later land over Q0 and Q1
+//   [32K, 48K) A (fp32, Sw64), then T in place, then T' hi and lo boxes
+//   [48K, 52K) A's diagonal blocks (diag_index), then scratch of the solve
+constexpr uint32_t P_KQ = 0, P_AT = 4 * SLOT, P_AD = 6 * SLOT, P_ALPHA = P_AD + 4096, P_BAR = P_ALPHA + 256;
+constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;  // + barriers, TMEM slot, abort flag; + alignment slack
+constexpr uint32_t P_TMEM_COLS = 128;           // G, then W^T (columns 0-63) and U^T (64-127)
+constexpr uint32_t ID_G = ptx::idesc_bf16(128, 64, false, false);     // [K; Q] K^T
+constexpr uint32_t ID_WU = ptx::idesc_bf16(128, 64, true, false);     // K^T T'^T, V^T T'^T
 
 // Byte offset of element (r, c) in a 64-column bf16 box with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw128_elem(int r, int c) {
     return (uint32_t)r * 128u + ((((uint32_t)c >> 3) ^ ((uint32_t)r & 7u)) << 4) + ((uint32_t)c & 7u) * 2u;
 }
 
-// Row tile i and column tile j (16 x 8 tiles of a 64 x 64 matrix) of tile
-// number idx: 0..19 are the tiles on or below the diagonal 16 x 16 blocks
-// (row by row), 20..31 the tiles above them.
-__device__ __forceinline__ void tile_ij(int idx, int &i, int &j) {
-    if (idx < 20) {
-        i = idx < 2 ? 0 : idx < 6 ? 1 : idx < 12 ? 2 : 3;
-        j = idx - i * (i + 1);
-    } else {
-        const int u = idx - 20;
-        i = u < 6 ? 0 : u < 10 ? 1 : 2;
-        j = i == 0 ? 2 + u : i == 1 ? u - 2 : u - 4;
-    }
-}
-
 // Everything about one chunk that does not depend on the state, written as
 // the workspace image chunk_tc_kernel reads (rows past L are zero):
-//   alpha = gate(beta, ||k||^2),  A = strictly-lower(diag(alpha) K K^T),
-//   T = (I + A)^{-1},  T' = T diag(alpha),
-//   -W = -T' K  (bf16),  M = lower-incl-diag(Q K^T)  (bf16),
-//   U = T' V  (fp32).
-// Products run on mma.sync with fp32 accumulation: bf16 q/k/v operands, T' as
-// a bf16 hi + lo pair, TF32 in the block rows of T.  One 256-thread CTA per
-// (b, h, chunk): independent chunks, so their latency overlaps across CTAs.
-__global__ void __launch_bounds__(kPrepThreads) chunk_prep_tc_kernel(const __nv_bfloat16 *__restrict__ q,
-                                                                     const __nv_bfloat16 *__restrict__ k,
-                                                                     const __nv_bfloat16 *__restrict__ v,
+//   alpha = gate(beta, ||k||^2)
+//   G = [K; Q] K^T                      (tcgen05: A = [K; Q], B = K)
+//   A = strictly-lower(diag(alpha) K K^T),  M = lower-incl-diag(Q K^T)  (bf16)
+//   T = (I + A)^{-1},  T' = T diag(alpha)   (CUDA cores + mma.sync TF32)
+//   W^T = K^T T'^T,  U^T = V^T T'^T     (tcgen05: A = K^T / V^T, B = T' as bf16 hi + lo)
+//   -> -W (bf16), U (fp32)
+// One 256-thread CTA per (b, h, chunk); thread 0 issues the TMA loads and the
+// tcgen05 products, all eight warps share the TMEM read-outs and the solve.
+__global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                     const __grid_constant__ CUtensorMap tm_k,
+                                                                     const __grid_constant__ CUtensorMap tm_v,
                                                                      const float *__restrict__ beta,
                                                                      unsigned char *__restrict__ ws, int L, int nc,
                                                                      int euler) {
-    extern __shared__ __align__(16) unsigned char psm_raw[];
-    PrepSmem &sm = *reinterpret_cast<PrepSmem *>(psm_raw);
-    const int p = threadIdx.x, w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
+    using namespace ptx;
+    extern __shared__ unsigned char psm_raw[];
+    unsigned char *sm =
+        reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(psm_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    float *alpha = reinterpret_cast<float *>(sm + P_ALPHA);
+    float *Ad = reinterpret_cast<float *>(sm + P_AD);
+    const Sw64 AT{reinterpret_cast<float *>(sm + P_AT)};
+    // barriers 0: K, Q landed  1: V landed  2: G done  3: W, U done  4: drain
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_BAR + 40);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + P_BAR + 44);
+    const int p = threadIdx.x, w = p >> 5, lane = p & 31;
     const long gidx = blockIdx.x;
     const int chunk = (int)(gidx % nc);
     const long bh = gidx / nc;
     const int t0 = chunk * C, n = min(C, L - t0);
     const size_t row0 = (size_t)bh * L + t0;
-#pragma unroll
-    for (int it = 0; it < C * (DK / 8) / kPrepThreads; ++it) {
-        const int e = p + kPrepThreads * it, r = e >> 4, c8 = (e & 15) * 8;
-        const bool ok = r < n;
-        const size_t go = (row0 + (ok ? r : 0)) * DK + c8;
-        cp_async16(&sm.K[r][c8], k + go, ok);
-        cp_async16(&sm.Q[r][c8], q + go, ok);
-        cp_async16(&sm.V[r][c8], v + go, ok);
+    if (p == 0) EFLA_TR(49, 1023);
+    if (p == 0) {
+        *abort_flag = 0;
+        for (int i = 0; i < 5; ++i) mbar_init(&bar[i], 1);
+        fence_mbar_init();
+        tma_prefetch(&tm_q);
+        tma_prefetch(&tm_k);
+        tma_prefetch(&tm_v);
+        mbar_expect_tx(&bar[0], 4 * SLOT);
+        tma_load_3d(sm + P_KQ, &tm_k, &bar[0], 0, t0, (int)bh);
+        tma_load_3d(sm + P_KQ + SLOT, &tm_q, &bar[0], 0, t0, (int)bh);
+        tma_load_3d(sm + P_KQ + 2 * SLOT, &tm_k, &bar[0], 64, t0, (int)bh);
+        tma_load_3d(sm + P_KQ + 3 * SLOT, &tm_q, &bar[0], 64, t0, (int)bh);
     }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    if (w == 0) {
+        tmem_alloc(tmem_slot, P_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    {   // gate: four lanes per key row
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // bounded wait by every thread; the answer is block-uniform
+    auto wait_all = [&](int i, uint32_t parity) { return !__syncthreads_or(!mbar_wait(&bar[i], parity, abort_flag)); };
+    bool issued_v = false, issued_mma = false;  // (thread 0) for the drain after a failure
+    bool ok = wait_all(0, 0);
+    if (p == 0) EFLA_TR(50, 1023);
+    if (p == 0 && ok) {  // G = [K; Q] K^T: 8 k-steps over d_k
+        tc_fence_after();
+        const uint64_t d0 = sdesc_sw128(sbase + P_KQ, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t d = d0 + (((kk >> 2) * 2 * SLOT + (kk & 3) * 32) >> 4);
+            mma_bf16(tmem, d, d, ID_G, kk > 0);
+        }
+        mma_commit(&bar[2]);
+        issued_mma = true;
+    }
+    if (ok) {   // gate from the K tile: four lanes per key row; 16-byte chunk c of
+                // row r sits in box c / 8 at position (c % 8) ^ (r % 8)
         const int r = p >> 2, h = p & 3;
         float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+            const int c = 4 * h + j;
             float f[8];
-            unpack8(*reinterpret_cast<const uint4 *>(&sm.K[r][32 * h + 8 * j]), f);
+            unpack8(*reinterpret_cast<const uint4 *>(sm + P_KQ + (c >> 3) * 2 * SLOT + sw128_chunk(r, c & 7)), f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc8[e] = fmaf(f[e], f[e], acc8[e]);
         }
         float ss = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
         ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-        if (h == 0) sm.alpha[r] = (r < n) ? gate_alpha(beta[row0 + r], ss, euler != 0) : 0.f;
+        if (h == 0) alpha[r] = (r < n) ? gate_alpha(beta[row0 + r], ss, euler != 0) : 0.f;
     }
-    __syncthreads();
+    ok = ok && wait_all(2, 0);  // (also publishes alpha)
+    tc_fence_after();
+    if (p == 0 && ok) {  // Q is no longer read: V lands over it while T is solved
+        mbar_expect_tx(&bar[1], 2 * SLOT);
+        tma_load_3d(sm + P_KQ + SLOT, &tm_v, &bar[1], 0, t0, (int)bh);
+        tma_load_3d(sm + P_KQ + 3 * SLOT, &tm_v, &bar[1], 64, t0, (int)bh);
+        issued_v = true;
+    }
     unsigned char *out = ws + (size_t)gidx * PREP_BYTES;
-    const Sw64 Af{sm.A}, Tf{sm.T};
-    // A (from K K^T) and M (from Q K^T) on the tiles on or below the diagonal
-    // blocks; M's other tiles are zero.  A's diagonal blocks go to Ad, the
-    // blocks left of them to Af.
-#pragma unroll 1
-    for (int idx = w; idx < 32; idx += kPrepThreads / 32) {
-        int i, j;
-        tile_ij(idx, i, j);
-        const int r0 = 16 * i + g, r1 = r0 + 8, c0 = 8 * j + 2 * t;
-        float qk[4] = {0.f, 0.f, 0.f, 0.f};
-        if (idx < 20) {
-            float kk[4] = {0.f, 0.f, 0.f, 0.f};
-            gram2_tile(sm.K, sm.Q, 16 * i, 8 * j, lane, kk, qk);
-            const float a00 = (c0 < r0) ? sm.alpha[r0] * kk[0] : 0.f, a01 = (c0 + 1 < r0) ? sm.alpha[r0] * kk[1] : 0.f;
-            const float a10 = (c0 < r1) ? sm.alpha[r1] * kk[2] : 0.f, a11 = (c0 + 1 < r1) ? sm.alpha[r1] * kk[3] : 0.f;
-            if ((j >> 1) == i) {  // diagonal block: column m = c - 16 i, row 2 s + h = r - 16 i
-                const int m = c0 - 16 * i, s0 = g >> 1, h = g & 1;
-                sm.Ad[diag_index(i, m, h, s0)] = a00;
-                sm.Ad[diag_index(i, m + 1, h, s0)] = a01;
-                sm.Ad[diag_index(i, m, h, s0 + 4)] = a10;
-                sm.Ad[diag_index(i, m + 1, h, s0 + 4)] = a11;
-            } else {
-                *reinterpret_cast<float2 *>(Af.at(r0, c0)) = make_float2(a00, a01);
-                *reinterpret_cast<float2 *>(Af.at(r1, c0)) = make_float2(a10, a11);
+    const int quad = w & 3, cpart = w >> 2;
+    if (ok) {
+        // G read-out: lanes 0-63 hold K K^T rows (-> A and its diagonal-block
+        // copy), lanes 64-127 Q K^T rows (-> M); warp (quad, cpart) takes
+        // columns 32 cpart .. + 31
+        uint32_t r32[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * cpart, r32);
+        tmem_ld_wait(r32);
+        if (quad < 2) {
+            const int i = 32 * quad + lane;
+            const float ai = alpha[i];
+#pragma unroll
+            for (int x = 0; x < 32; x += 2) {
+                const int j = 32 * cpart + x;
+                const float a0 = (j < i) ? ai * __uint_as_float(r32[x]) : 0.f;
+                const float a1 = (j + 1 < i) ? ai * __uint_as_float(r32[x + 1]) : 0.f;
+                if ((j >> 4) == (i >> 4)) {
+                    const int b = i >> 4, m = j & 15, rl = i & 15;
+                    Ad[diag_index(b, m, rl & 1, rl >> 1)] = a0;
+                    Ad[diag_index(b, m + 1, rl & 1, rl >> 1)] = a1;
+                } else if ((j >> 4) < (i >> 4)) {
+                    *reinterpret_cast<float2 *>(AT.at(i, j)) = make_float2(a0, a1);
+                }
+            }
+        } else {
+            const int i = 32 * (quad - 2) + lane;
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                uint32_t v4[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int x = 8 * c8 + 2 * u, j = 32 * cpart + x;
+                    v4[u] = pack_bf16((j <= i) ? __uint_as_float(r32[x]) : 0.f,
+                                      (j + 1 <= i) ? __uint_as_float(r32[x + 1]) : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(out + IMG_M + sw128_elem(i, 32 * cpart + 8 * c8)) =
+                    make_uint4(v4[0], v4[1], v4[2], v4[3]);
             }
         }
-        *reinterpret_cast<uint32_t *>(out + IMG_M + sw128_elem(r0, c0)) =
-            ptx::pack_bf16((c0 <= r0) ? qk[0] : 0.f, (c0 + 1 <= r0) ? qk[1] : 0.f);
-        *reinterpret_cast<uint32_t *>(out + IMG_M + sw128_elem(r1, c0)) =
-            ptx::pack_bf16((c0 <= r1) ? qk[2] : 0.f, (c0 + 1 <= r1) ? qk[3] : 0.f);
     }
-    __syncthreads();  // Q is dead from here; its space becomes T
-    invert_unit_lower<kPrepThreads>(p, sm.Ad, Af, Tf);
-    // T' = T diag(alpha) (lower triangle) as swizzled bf16 hi and lo boxes in A's space
-#pragma unroll
-    for (int it = 0; it < 2; ++it) {
-        const int e = p + kPrepThreads * it, r = e >> 3, jj = e & 7;
-        const float4 ta = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * jj));
-        const float4 tb = *reinterpret_cast<const float4 *>(Tf.at(r, 8 * jj + 4));
-        const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
-        uint32_t h4[4], l4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int c = 8 * jj + 2 * u;
-            split2((c <= r) ? tv[2 * u] * sm.alpha[c] : 0.f, (c + 1 <= r) ? tv[2 * u + 1] * sm.alpha[c + 1] : 0.f,
-                   h4[u], l4[u]);
-        }
-        *reinterpret_cast<uint4 *>(sm.TP[0] + ptx::sw128_chunk(r, jj)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-        *reinterpret_cast<uint4 *>(sm.TP[1] + ptx::sw128_chunk(r, jj)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
-    }
+    tc_fence_before();
     __syncthreads();
-    // -W = -T' K and U = T' V: warp w owns the 8-column tiles 2w and 2w+1 of
-    // both, for all four 16-row tiles; T' is lower triangular, so row tile i
-    // needs k < 16 (i + 1).  ldmatrix lane l addresses row (l & 7) + 8 ((l >> 3) & 1)
-    // of the 16-row block and 8-column group (l >> 4).
-    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lgrp = lane >> 4;
-#pragma unroll 1
-    for (int i = 0; i < 4; ++i) {
-        float aw[2][4], au[2][4];
+    if (p == 0) EFLA_TR(51, 1023);
+    if (ok) {
+        invert_unit_lower<kPrepThreads>(p, Ad, AT);
+        if (p == 0) EFLA_TR(52, 1023);
+        // T' = T diag(alpha) (lower triangle) as 128-byte-swizzled bf16 hi and
+        // lo boxes (rows i, 64 columns j: the K-major B operand T'^T), written
+        // over T once every thread holds its part of T
+        float tv[2][8];
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) aw[u][e] = au[u][e] = 0.f;
-        const int ar = 16 * i + lrow;
-#pragma unroll 1
-        for (int k0 = 0; k0 < 16 * (i + 1); k0 += 16) {
-            uint32_t ah[4], al[4], bk0[2], bk1[2], bv0[2], bv1[2];
-            const uint32_t aoff = ptx::sw128_chunk(ar, (k0 >> 3) + lgrp);
-            ldsm_x4(sm.TP[0] + aoff, ah);
-            ldsm_x4(sm.TP[1] + aoff, al);
-            ldsm_x4t(&sm.K[k0 + lrow][8 * (2 * w + lgrp)], bk0, bk1);
-            ldsm_x4t(&sm.V[k0 + lrow][8 * (2 * w + lgrp)], bv0, bv1);
-            mma_bf16_16816(aw[0], ah, bk0);
-            mma_bf16_16816(aw[1], ah, bk1);
-            mma_bf16_16816(au[0], ah, bv0);
-            mma_bf16_16816(au[1], ah, bv1);
-            mma_bf16_16816(aw[0], al, bk0);
-            mma_bf16_16816(aw[1], al, bk1);
-            mma_bf16_16816(au[0], al, bv0);
-            mma_bf16_16816(au[1], al, bv1);
+        for (int it = 0; it < 2; ++it) {
+            const int e = p + kPrepThreads * it, r = e >> 3, jj = e & 7;
+            const float4 ta = *reinterpret_cast<const float4 *>(AT.at(r, 8 * jj));
+            const float4 tb = *reinterpret_cast<const float4 *>(AT.at(r, 8 * jj + 4));
+            tv[it][0] = ta.x, tv[it][1] = ta.y, tv[it][2] = ta.z, tv[it][3] = ta.w;
+            tv[it][4] = tb.x, tv[it][5] = tb.y, tv[it][6] = tb.z, tv[it][7] = tb.w;
         }
+        __syncthreads();
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int c = 8 * (2 * w + u) + 2 * t;  // d column, 0..127
-            const int box = c >> 6, cc = c & 63;
+        for (int it = 0; it < 2; ++it) {
+            const int e = p + kPrepThreads * it, r = e >> 3, jj = e & 7;
+            uint32_t h4[4], l4[4];
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int r = 16 * i + g + 8 * hr;
-                *reinterpret_cast<uint32_t *>(out + IMG_W + box * SLOT + sw128_elem(r, cc)) =
-                    ptx::pack_bf16(-aw[u][2 * hr], -aw[u][2 * hr + 1]);
-                const uint32_t uo =
-                    IMG_U + box * UHALF + r * 256 + ((((uint32_t)cc >> 2) ^ ((uint32_t)r & 15u)) << 4) + (cc & 3) * 4;
-                *reinterpret_cast<float2 *>(out + uo) = make_float2(au[u][2 * hr], au[u][2 * hr + 1]);
+            for (int u = 0; u < 4; ++u) {
+                const int c = 8 * jj + 2 * u;
+                split2((c <= r) ? tv[it][2 * u] * alpha[c] : 0.f, (c + 1 <= r) ? tv[it][2 * u + 1] * alpha[c + 1] : 0.f,
+                       h4[u], l4[u]);
             }
+            *reinterpret_cast<uint4 *>(sm + P_AT + sw128_chunk(r, jj)) = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+            *reinterpret_cast<uint4 *>(sm + P_AT + SLOT + sw128_chunk(r, jj)) = make_uint4(l4[0], l4[1], l4[2], l4[3]);
         }
+        fence_proxy_async();
+    }
+    if (p == 0) EFLA_TR(53, 1023);
+    ok = ok && wait_all(1, 0);  // (also orders the T' image before the products)
+    if (p == 0 && ok) {  // W^T = K^T (T'_hi + T'_lo)^T, U^T = V^T (...)^T: 4 k-steps over the chunk, hi and lo
+        tc_fence_after();
+        const uint64_t dK = sdesc_sw128(sbase + P_KQ, 2 * SLOT, 1024);
+        const uint64_t dV = sdesc_sw128(sbase + P_KQ + SLOT, 2 * SLOT, 1024);
+        const uint64_t dT = sdesc_sw128(sbase + P_AT, 16, 1024);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t b = dT + ((part * SLOT + kk * 32) >> 4);
+                mma_bf16(tmem, dK + ((kk * 2048) >> 4), b, ID_WU, part | kk);
+                mma_bf16(tmem + 64, dV + ((kk * 2048) >> 4), b, ID_WU, part | kk);
+            }
+        mma_commit(&bar[3]);
+    }
+    ok = ok && wait_all(3, 0);
+    tc_fence_after();
+    if (ok) {
+        // W^T, U^T read-out: lane d (d_k for W, d_v for U), columns i = chunk rows
+        // 32 cpart .. + 31 -> -W[i][d] (bf16 box d / 64) and U[i][d] (fp32 half d / 64)
+        const int d = 32 * quad + lane, box = d >> 6, dc = d & 63;
+        uint32_t r32[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * cpart, r32);
+        tmem_ld_wait(r32);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+            const int i = 32 * cpart + x;
+            *reinterpret_cast<__nv_bfloat16 *>(out + IMG_W + box * SLOT + sw128_elem(i, dc)) =
+                __float2bfloat16_rn(-__uint_as_float(r32[x]));
+        }
+        tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 64 + 32 * cpart, r32);
+        tmem_ld_wait(r32);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+            const int i = 32 * cpart + x;
+            *reinterpret_cast<uint32_t *>(out + IMG_U + box * UHALF + i * 256 +
+                                          ((((uint32_t)dc >> 2) ^ ((uint32_t)i & 15u)) << 4) + (dc & 3) * 4) = r32[x];
+        }
+    }
+    if (p == 0) EFLA_TR(54, 1023);
+    if (p == 0 && !ok) {
+        // after a failed wait: every TMA load issued lands and every product
+        // completes before the CTA exits (bounded waits that ignore the abort)
+        int never = 0;
+        mbar_wait(&bar[0], 0, &never);
+        if (issued_v) mbar_wait(&bar[1], 0, &never);
+        if (issued_mma) {
+            mma_commit(&bar[4]);
+            mbar_wait(&bar[4], 0, &never);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (w == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, P_TMEM_COLS);
     }
 }
 
@@ -932,15 +936,16 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
         !make_map(&mo, o, bh, L, of32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                   (int)sizeof(Tout), of32 ? 32u : 64u))
         return EFLA_ERR_CUDA;
-    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES) || !ensure_smem<chunk_prep_tc_kernel>(sizeof(PrepSmem)))
+    CUtensorMap mv;
+    if (!make_map_bf16_sw128(&mv, v, bh, L)) return EFLA_ERR_CUDA;
+    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES) || !ensure_smem<chunk_prep_tc_kernel>(P_SMEM))
         return EFLA_ERR_CUDA;
     const long grid = bh * NSPLIT;
     const int nc = (L + C - 1) / C;
     if (grid > 0x7fffffffL || bh * nc > 0x7fffffffL) return EFLA_ERR_SHAPE;
     unsigned char *img = static_cast<unsigned char *>(ws);
-    chunk_prep_tc_kernel<<<(unsigned)(bh * nc), kPrepThreads, sizeof(PrepSmem), st>>>(
-        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-        static_cast<const __nv_bfloat16 *>(v), beta, img, L, nc, euler ? 1 : 0);
+    chunk_prep_tc_kernel<<<(unsigned)(bh * nc), kPrepThreads, P_SMEM, st>>>(mq, mk, mv, beta, img, L, nc,
+                                                                            euler ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
     chunk_tc_kernel<Tout><<<(unsigned)grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mo, img, S0, SL, L, nc);
     return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
