@@ -60,8 +60,9 @@ __global__ void __launch_bounds__(256, 1) chunk_prep_kernel(const Tin *__restric
     PrepSmem<D> &sm = *reinterpret_cast<PrepSmem<D> *>(smem_raw);
     constexpr int LD = PrepSmem<D>::LD, LC = PrepSmem<D>::LC, C = kChunk;
     const int t = threadIdx.x;
-    const int chunk = blockIdx.x % n_chunks;
-    const long bh = blockIdx.x / n_chunks;
+    const unsigned q32 = blockIdx.x / (unsigned)n_chunks;  // 32-bit division: grid < 2^31
+    const int chunk = (int)(blockIdx.x - q32 * (unsigned)n_chunks);
+    const long bh = (long)q32;
     const int t0 = chunk * C;
     const int n = min(C, L - t0);
     const long row0 = bh * (long)L + t0;

@@ -180,7 +180,7 @@ struct Sw64 {
 __device__ __forceinline__ int diag_index(int b, int m, int h, int s) { return ((b * 16 + m) * 2 + h) * 8 + s; }
 
 // T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A, in place:
-// AT holds A's blocks left of the diagonal on entry and T's lower triangle
+// AT holds A's blocks left of the diagonal (rounded to TF32) on entry and T's lower triangle
 // (diagonal blocks included) on return.  First the four 16 x 16 diagonal
 // blocks by right-looking forward substitution (warps 0-3, one block each,
 // one column per lane pair, fp32, A's diagonal blocks read from their own
@@ -226,8 +226,10 @@ __device__ __forceinline__ void invert_unit_lower(const int p, float *__restrict
             // R tile = A[r0.., k] T[k, c0..] over k from the column's own block up to r0
 #pragma unroll 1
             for (int k0 = 16 * (w >> 1); k0 < r0; k0 += 8) {
-                const uint32_t a[4] = {f2tf32(*AT.at(r0 + g, k0 + t)), f2tf32(*AT.at(r0 + g + 8, k0 + t)),
-                                       f2tf32(*AT.at(r0 + g, k0 + t + 4)), f2tf32(*AT.at(r0 + g + 8, k0 + t + 4))};
+                // A's tiles are stored already rounded to TF32
+                const uint32_t a[4] = {__float_as_uint(*AT.at(r0 + g, k0 + t)), __float_as_uint(*AT.at(r0 + g + 8, k0 + t)),
+                                       __float_as_uint(*AT.at(r0 + g, k0 + t + 4)),
+                                       __float_as_uint(*AT.at(r0 + g + 8, k0 + t + 4))};
                 const uint32_t bb[2] = {f2tf32(*AT.at(k0 + t, c0 + g)), f2tf32(*AT.at(k0 + t + 4, c0 + g))};
                 mma_tf32(acc, a, bb);
             }
@@ -305,6 +307,14 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until every committed bulk store of this thread has completed.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// cp.async.bulk shared -> global of `bytes` (multiple of 16, both ends
+// 16-byte aligned), in this thread's bulk async group.
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+                 "r"(ptx::smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
 
 // Bounded wait by a whole warp; the answer is warp-uniform (false when any lane gave up).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
@@ -637,6 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------- prep kernel
 constexpr int kPrepThreads = 256;
+constexpr int kCopyThread = 224;  // lane 0 of warp 7, idle during the diagonal solves
 // Shared memory of one prep CTA (base aligned to 1024 B):
 //   [0, 32K)   K0 Q0 K1 Q1 (64 x 64 bf16 boxes, 128-byte swizzle): [K; Q] is
 //              the 128-row A operand of [K; Q] K^T per d_k half, K also its B;
@@ -645,9 +656,12 @@ constexpr int kPrepThreads = 256;
 //   [48K, 52K) A's diagonal blocks (diag_index), then scratch of the solve
 constexpr uint32_t P_KQ = 0, P_AT = 4 * SLOT, P_AD = 6 * SLOT, P_ALPHA = P_AD + 4096, P_BAR = P_ALPHA + 256;
 constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;  // + barriers, TMEM slot, abort flag; + alignment slack
-constexpr uint32_t P_TMEM_COLS = 128;           // G, then W^T (columns 0-63) and U^T (64-127)
-constexpr uint32_t ID_G = ptx::idesc_bf16(128, 64, false, false);     // [K; Q] K^T
-constexpr uint32_t ID_WU = ptx::idesc_bf16(128, 64, true, false);     // K^T T'^T, V^T T'^T
+constexpr uint32_t P_TMEM_COLS = 128;           // G (columns 0-63), then W, then U (0-127)
+constexpr uint32_t ID_G = ptx::idesc_bf16(128, 64, false, false);  // [K; Q] K^T
+// T' K and T' V: M = 64 (T' rows), N = 128, B MN-major.  An M = 64
+// accumulator keeps row i in TMEM lane (i % 16) + 32 (i / 16), its N
+// columns contiguous (the first 16 lanes of each warp's 32-lane quarter).
+constexpr uint32_t ID_WU = ptx::idesc_bf16(64, 128, false, true);
 
 // Byte offset of element (r, c) in a 64-column bf16 box with the 128-byte swizzle.
 __device__ __forceinline__ uint32_t sw128_elem(int r, int c) {
@@ -660,7 +674,7 @@ __device__ __forceinline__ uint32_t sw128_elem(int r, int c) {
 //   G = [K; Q] K^T                      (tcgen05: A = [K; Q], B = K)
 //   A = strictly-lower(diag(alpha) K K^T),  M = lower-incl-diag(Q K^T)  (bf16)
 //   T = (I + A)^{-1},  T' = T diag(alpha)   (CUDA cores + mma.sync TF32)
-//   W^T = K^T T'^T,  U^T = V^T T'^T     (tcgen05: A = K^T / V^T, B = T' as bf16 hi + lo)
+//   W = T' K,  U = T' V                 (tcgen05, M = 64: A = T' as bf16 hi + lo, B = K / V)
 //   -> -W (bf16), U (fp32)
 // One 256-thread CTA per (b, h, chunk); thread 0 issues the TMA loads and the
 // tcgen05 products, all eight warps share the TMEM read-outs and the solve.
@@ -678,20 +692,23 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     float *alpha = reinterpret_cast<float *>(sm + P_ALPHA);
     float *Ad = reinterpret_cast<float *>(sm + P_AD);
     const Sw64 AT{reinterpret_cast<float *>(sm + P_AT)};
-    // barriers 0: K, Q landed  1: V landed  2: G done  3: W, U done  4: drain
+    // barriers 0: K, Q landed  1: V landed  2: G done  3: W done  4: U done  5: drain
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_BAR + 40);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + P_BAR + 44);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_BAR + 48);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + P_BAR + 52);
     const int p = threadIdx.x, w = p >> 5, lane = p & 31;
     const long gidx = blockIdx.x;
-    const int chunk = (int)(gidx % nc);
-    const long bh = gidx / nc;
+    // 32-bit quotient and remainder (grid < 2^31; a 64-bit division is a long
+    // instruction sequence on the slow conversion pipe)
+    const unsigned q32 = blockIdx.x / (unsigned)nc;
+    const int chunk = (int)(blockIdx.x - q32 * (unsigned)nc);
+    const long bh = (long)q32;
     const int t0 = chunk * C, n = min(C, L - t0);
     const size_t row0 = (size_t)bh * L + t0;
     if (p == 0) EFLA_TR(49, 1023);
     if (p == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < 5; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
         fence_mbar_init();
         tma_prefetch(&tm_q);
         tma_prefetch(&tm_k);
@@ -712,7 +729,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     const uint32_t tmem = *tmem_slot;
     // bounded wait by every thread; the answer is block-uniform
     auto wait_all = [&](int i, uint32_t parity) { return !__syncthreads_or(!mbar_wait(&bar[i], parity, abort_flag)); };
-    bool issued_v = false, issued_mma = false;  // (thread 0) for the drain after a failure
+    bool issued_v = false, issued_mma = false;  // (copy thread / thread 0) for the drain after a failure
     bool ok = wait_all(0, 0);
     if (p == 0) EFLA_TR(50, 1023);
     if (p == 0 && ok) {  // G = [K; Q] K^T: 8 k-steps over d_k
@@ -745,12 +762,6 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     }
     ok = ok && wait_all(2, 0);  // (also publishes alpha)
     tc_fence_after();
-    if (p == 0 && ok) {  // Q is no longer read: V lands over it while T is solved
-        mbar_expect_tx(&bar[1], 2 * SLOT);
-        tma_load_3d(sm + P_KQ + SLOT, &tm_v, &bar[1], 0, t0, (int)bh);
-        tma_load_3d(sm + P_KQ + 3 * SLOT, &tm_v, &bar[1], 64, t0, (int)bh);
-        issued_v = true;
-    }
     unsigned char *out = ws + (size_t)gidx * PREP_BYTES;
     const int quad = w & 3, cpart = w >> 2;
     if (ok) {
@@ -772,8 +783,9 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
                     const int b = i >> 4, m = j & 15, rl = i & 15;
                     Ad[diag_index(b, m, rl & 1, rl >> 1)] = a0;
                     Ad[diag_index(b, m + 1, rl & 1, rl >> 1)] = a1;
-                } else if ((j >> 4) < (i >> 4)) {
-                    *reinterpret_cast<float2 *>(AT.at(i, j)) = make_float2(a0, a1);
+                } else if ((j >> 4) < (i >> 4)) {  // only ever a TF32 operand: stored rounded
+                    *reinterpret_cast<float2 *>(AT.at(i, j)) =
+                        make_float2(__uint_as_float(f2tf32(a0)), __uint_as_float(f2tf32(a1)));
                 }
             }
         } else {
@@ -787,20 +799,32 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
                     v4[u] = pack_bf16((j <= i) ? __uint_as_float(r32[x]) : 0.f,
                                       (j + 1 <= i) ? __uint_as_float(r32[x + 1]) : 0.f);
                 }
-                *reinterpret_cast<uint4 *>(out + IMG_M + sw128_elem(i, 32 * cpart + 8 * c8)) =
+                // staged in the Q0 box (free once G is done), stored by one bulk copy
+                *reinterpret_cast<uint4 *>(sm + P_KQ + SLOT + sw128_elem(i, 32 * cpart + 8 * c8)) =
                     make_uint4(v4[0], v4[1], v4[2], v4[3]);
             }
         }
+        fence_proxy_async();
     }
     tc_fence_before();
     __syncthreads();
+    if (p == kCopyThread && ok) {
+        // M out; then V over Q (Q0 once M has been read out of it), landing while T is solved
+        bulk_store(out + IMG_M, sm + P_KQ + SLOT, SLOT);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_expect_tx(&bar[1], 2 * SLOT);
+        tma_load_3d(sm + P_KQ + SLOT, &tm_v, &bar[1], 0, t0, (int)bh);
+        tma_load_3d(sm + P_KQ + 3 * SLOT, &tm_v, &bar[1], 64, t0, (int)bh);
+        issued_v = true;
+    }
     if (p == 0) EFLA_TR(51, 1023);
     if (ok) {
         invert_unit_lower<kPrepThreads>(p, Ad, AT);
         if (p == 0) EFLA_TR(52, 1023);
         // T' = T diag(alpha) (lower triangle) as 128-byte-swizzled bf16 hi and
-        // lo boxes (rows i, 64 columns j: the K-major B operand T'^T), written
-        // over T once every thread holds its part of T
+        // lo boxes (rows i, 64 columns j: the K-major A operand), written over
+        // T once every thread holds its part of T
         float tv[2][8];
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
@@ -828,56 +852,97 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     }
     if (p == 0) EFLA_TR(53, 1023);
     ok = ok && wait_all(1, 0);  // (also orders the T' image before the products)
-    if (p == 0 && ok) {  // W^T = K^T (T'_hi + T'_lo)^T, U^T = V^T (...)^T: 4 k-steps over the chunk, hi and lo
+    // W = (T'_hi + T'_lo) K, then U = (T'_hi + T'_lo) V in the same columns:
+    // 4 k-steps over the chunk, hi and lo; B = the K or V tile, MN-major
+    // (d columns 0-63 and 64-127 two swizzled boxes apart)
+    auto issue_wu = [&](uint32_t tile, int done) {
         tc_fence_after();
-        const uint64_t dK = sdesc_sw128(sbase + P_KQ, 2 * SLOT, 1024);
-        const uint64_t dV = sdesc_sw128(sbase + P_KQ + SLOT, 2 * SLOT, 1024);
+        const uint64_t dB = sdesc_sw128(sbase + P_KQ + tile, 2 * SLOT, 1024);
         const uint64_t dT = sdesc_sw128(sbase + P_AT, 16, 1024);
 #pragma unroll
         for (int part = 0; part < 2; ++part)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t b = dT + ((part * SLOT + kk * 32) >> 4);
-                mma_bf16(tmem, dK + ((kk * 2048) >> 4), b, ID_WU, part | kk);
-                mma_bf16(tmem + 64, dV + ((kk * 2048) >> 4), b, ID_WU, part | kk);
-            }
-        mma_commit(&bar[3]);
-    }
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem, dT + ((part * SLOT + kk * 32) >> 4), dB + ((kk * 2048) >> 4), ID_WU, part | kk);
+        mma_commit(&bar[done]);
+    };
+    // row i of W / U sits in TMEM lane (i % 16) + 32 (i / 16): warp (quad,
+    // cpart) lanes 0-15 hold rows 16 quad + lane, columns 64 cpart .. + 63
+    // (= the bf16 box / fp32 half cpart of the image)
+    const int wrow = 16 * quad + (lane & 15);
+    const bool wlane = lane < 16;
+    const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16) + 64 * cpart;
+    if (p == 0 && ok) issue_wu(0, 3);
     ok = ok && wait_all(3, 0);
     tc_fence_after();
     if (ok) {
-        // W^T, U^T read-out: lane d (d_k for W, d_v for U), columns i = chunk rows
-        // 32 cpart .. + 31 -> -W[i][d] (bf16 box d / 64) and U[i][d] (fp32 half d / 64)
-        const int d = 32 * quad + lane, box = d >> 6, dc = d & 63;
-        uint32_t r32[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * cpart, r32);
-        tmem_ld_wait(r32);
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-            const int i = 32 * cpart + x;
-            *reinterpret_cast<__nv_bfloat16 *>(out + IMG_W + box * SLOT + sw128_elem(i, dc)) =
-                __float2bfloat16_rn(-__uint_as_float(r32[x]));
-        }
-        tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 64 + 32 * cpart, r32);
-        tmem_ld_wait(r32);
+        for (int h = 0; h < 2; ++h) {  // 32 columns at a time
+            uint32_t r32[32];
+            tmem_ld32(tq + 32 * h, r32);
+            tmem_ld_wait(r32);
+            if (wlane) {  // staged in the K box of the same d_k half (K is no longer read)
+                unsigned char *dst = sm + P_KQ + cpart * 2 * SLOT + wrow * 128;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-            const int i = 32 * cpart + x;
-            *reinterpret_cast<uint32_t *>(out + IMG_U + box * UHALF + i * 256 +
-                                          ((((uint32_t)dc >> 2) ^ ((uint32_t)i & 15u)) << 4) + (dc & 3) * 4) = r32[x];
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v4[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        v4[u] = pack_bf16(-__uint_as_float(r32[8 * c + 2 * u]), -__uint_as_float(r32[8 * c + 2 * u + 1]));
+                    *reinterpret_cast<uint4 *>(dst + (((4 * h + c) ^ (wrow & 7)) << 4)) =
+                        make_uint4(v4[0], v4[1], v4[2], v4[3]);
+                }
+            }
         }
     }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (p == 0 && ok) {
+        bulk_store(out + IMG_W, sm + P_KQ, SLOT);
+        bulk_store(out + IMG_W + SLOT, sm + P_KQ + 2 * SLOT, SLOT);
+        bulk_commit();
+        issue_wu(SLOT, 4);
+        bulk_wait_read0();  // the K boxes are reused for U below
+    }
+    ok = ok && wait_all(4, 0);
+    tc_fence_after();
+    if (ok) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t r32[32];
+            tmem_ld32(tq + 32 * h, r32);
+            tmem_ld_wait(r32);
+            if (wlane) {  // staged: half 0 over T', half 1 over the K0 and V0 boxes
+                unsigned char *dst = sm + (cpart ? P_KQ : P_AT) + wrow * 256;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(dst + (((8 * h + c) ^ (wrow & 15)) << 4)) =
+                        make_uint4(r32[4 * c], r32[4 * c + 1], r32[4 * c + 2], r32[4 * c + 3]);
+            }
+        }
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (p == 0 && ok) {
+        bulk_store(out + IMG_U, sm + P_AT, UHALF);
+        bulk_store(out + IMG_U + UHALF, sm + P_KQ, UHALF);
+        bulk_commit();
+    }
+    if (p == 0 || p == kCopyThread) bulk_wait0();  // the image is written before the CTA exits
     if (p == 0) EFLA_TR(54, 1023);
-    if (p == 0 && !ok) {
+    if (!ok) {
         // after a failed wait: every TMA load issued lands and every product
         // completes before the CTA exits (bounded waits that ignore the abort)
         int never = 0;
-        mbar_wait(&bar[0], 0, &never);
-        if (issued_v) mbar_wait(&bar[1], 0, &never);
-        if (issued_mma) {
-            mma_commit(&bar[4]);
-            mbar_wait(&bar[4], 0, &never);
+        if (p == 0) {
+            mbar_wait(&bar[0], 0, &never);
+            if (issued_mma) {
+                mma_commit(&bar[5]);
+                mbar_wait(&bar[5], 0, &never);
+            }
         }
+        if (p == kCopyThread && issued_v) mbar_wait(&bar[1], 0, &never);
     }
     tc_fence_before();
     __syncthreads();
