@@ -321,11 +321,27 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort));
 }
 
+// One run of the serial kernel over a contiguous range of chunks, for every
+// (b, h, d_v half) of the grid: the whole sequence, or one segment of it.
+struct SegJob {
+    int c0, nch;      // first chunk and number of chunks
+    int s0_kind;      // initial state: 0 zero, 1 read from s0, 2 the identity
+    int write_o;      // store the outputs of these chunks
+    const float *s0;  // [B*H][d_k][d_v] fp32 (s0_kind 1)
+    float *sl;        // final state, [B*H][d_k][d_v] fp32, or null
+};
+constexpr int kMaxJobs = 16;
+// The jobs of one launch (blockIdx.y picks the job) and the sequence's chunk count.
+struct SegPlan {
+    int nc, njobs;
+    SegJob job[kMaxJobs];
+};
+
 template <typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_o, const unsigned char *__restrict__ ws,
-                    const float *__restrict__ S0, float *__restrict__ SL, int L, int nc) {
+                    const __grid_constant__ SegPlan plan) {
     using namespace ptx;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm =
@@ -338,6 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long bh = blockIdx.x / NSPLIT;
     const int half = blockIdx.x % NSPLIT, j0 = half * DVT;
+    const SegJob &job = plan.job[blockIdx.y];
+    const int nc = plan.nc, cb = job.c0, ncj = job.nch;  // chunks cb .. cb + ncj - 1 of nc
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -374,8 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
         const bool dwarp = quad >= 2;  // lanes 64..127: the D rows of Y
         float x[32];
-        {   // initial state
-            const float *src = S0 ? S0 + ((size_t)bh * DK + row) * DK + j0 + c0 : nullptr;
+        {   // initial state: zero, given, or the identity (columns j0 + c0 .. of row `row`)
+            const float *src = job.s0_kind == 1 ? job.s0 + ((size_t)bh * DK + row) * DK + j0 + c0 : nullptr;
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
                 const float4 v = src ? *reinterpret_cast<const float4 *>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -383,6 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 x[c + 1] = v.y;
                 x[c + 2] = v.z;
                 x[c + 3] = v.w;
+            }
+            if (job.s0_kind == 2) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) x[c] = (row == j0 + c0 + c) ? 1.f : 0.f;
             }
             uint32_t r[32];
 #pragma unroll
@@ -397,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Only the 256-thread vote on barrier 2 leaves the loop: a failed wait
         // inside one group (barriers 1 and 3) skips that group's work, and the
         // abort flag it set makes the next vote leave.
-        for (int n = 0; n < nc; ++n) {
+        for (int n = 0; n < ncj; ++n) {
             const int b = n & 1;
             const uint32_t ty = T_Y + 64 * b + c0;
             bool bad = false;
@@ -454,8 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bar[B_SBFULL]);
                 if (row == 64 && cpart == 0) EFLA_TR(13, n);
             }
-            if (n == nc - 1 && SL) {
-                float *dst = SL + ((size_t)bh * DK + row) * DK + j0 + c0;
+            if (n == ncj - 1 && job.sl) {
+                float *dst = job.sl + ((size_t)bh * DK + row) * DK + j0 + c0;
 #pragma unroll
                 for (int c = 0; c < 32; c += 4)
                     *reinterpret_cast<float4 *>(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
@@ -495,9 +517,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     fence_proxy_async();
                     named_bar(3, 128);
-                    if (storer) {
-                        tma_store_3d(&tm_o, sm + OFF_OST, j0, n * C, (int)bh);
-                        if constexpr (sizeof(Tout) == 4) tma_store_3d(&tm_o, sm + OFF_OST + SLOT, j0 + 32, n * C, (int)bh);
+                    if (storer && job.write_o) {
+                        tma_store_3d(&tm_o, sm + OFF_OST, j0, (cb + n) * C, (int)bh);
+                        if constexpr (sizeof(Tout) == 4)
+                            tma_store_3d(&tm_o, sm + OFF_OST + SLOT, j0 + 32, (cb + n) * C, (int)bh);
                         bulk_commit();
                     }
                 }
@@ -532,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bar[B_EMPTYB + b]);
         };
         int n = 0;
-        for (; n < nc; ++n) {
+        for (; n < ncj; ++n) {
             const int s = n & 1;
             const uint32_t sa = sbase + (uint32_t)s * STAGE, ty = tmem + T_Y + 64 * s;
             // Y = [Q; -W] (S_hi + S_lo) after: part A of the stage landed, O of
@@ -576,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
         }
-        if (n == nc && leader) issue_O(nc - 1);
+        if (n == ncj && leader) issue_O(ncj - 1);
         __syncwarp();
         // drain: wait (bounded, even after an abort) until every MMA issued has completed
         if (leader) mma_commit(&bar[B_DRAIN]);
@@ -593,11 +616,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const unsigned char *img = ws + (size_t)bh * nc * PREP_BYTES;
         int lastA[2] = {-1, -1}, lastB[2] = {-1, -1};  // last chunk loaded per stage and part
-        for (int n = 0; n < nc; ++n) {
+        for (int n = 0; n < ncj; ++n) {
             const int s = n & 1;
             unsigned char *st = sm + s * STAGE;
-            const int y = n * C, z = (int)bh;
-            const unsigned char *src = img + (size_t)n * PREP_BYTES;
+            const int y = (cb + n) * C, z = (int)bh;
+            const unsigned char *src = img + (size_t)(cb + n) * PREP_BYTES;
             // part A: Q and -W, once Y of chunk n-2 no longer reads them
             if (n >= 2 && !warp_wait(&bar[B_EMPTYA + s], ((n >> 1) - 1) & 1, abort_flag)) break;
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
@@ -990,7 +1013,91 @@ inline bool make_map_bf16_sw128(CUtensorMap *m, const void *base, long bh, int L
 }
 
 // Scratch of the tensor-core path: one -W / M / U image per chunk.
-inline size_t workspace_bytes(long bh, int L) { return (size_t)bh * ((L + C - 1) / C) * PREP_BYTES; }
+// Number of SMs of the current device (looked up once per device).
+inline int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+// Segment-parallel prefill for problems with too few heads to fill the GPU.
+// The sequence splits into P segments; the state map of segment r is affine,
+// S_out = M_r S_in + S_r, with S_r its final state from zero and M_r its final
+// state from the identity minus S_r.  Pass A runs, in one launch, segment 0
+// from the true S0 (with outputs) and every middle segment from 0 and from I;
+// a chain of small fp32 products then gives every segment's true initial
+// state, S_in(r+1) = M_r S_in(r) + S_r; pass B reruns segments 1..P-1 from
+// those with outputs.  Serial latency drops from nc to about 2 nc / P chunks.
+// P is the largest value in [3, 8] whose pass A (2 CTAs for segment 0, 4 for
+// each middle segment, per (b, h)) fits one wave, with at least
+// kMinSegChunks chunks per segment; otherwise 1 (a single pass).
+constexpr int kMinSegChunks = 16;
+inline int segments(long bh, int nc) {
+    const long sms = sm_count();
+    int best = 1;
+    for (int p = 3; p <= 8; ++p)
+        if (NSPLIT * bh * (1 + 2 * (p - 2)) <= sms && nc / p >= kMinSegChunks) best = p;
+    return best;
+}
+inline size_t state_bytes(long bh) { return (size_t)bh * DK * DK * sizeof(float); }
+
+// Scratch of the tensor-core path: one -W / M / U image per chunk, then (when
+// the prefill is segmented) 3P - 5 state buffers: S_in(1..P-1), the final
+// states of the middle segments from zero, and from the identity.
+inline size_t workspace_bytes(long bh, int L) {
+    const int nc = (L + C - 1) / C, P = segments(bh, nc);
+    return (size_t)bh * nc * PREP_BYTES + (P > 1 ? (size_t)(3 * P - 5) * state_bytes(bh) : 0);
+}
+
+// out = (SI - SZ) X + SZ for every (b, h): one step of the segment chain, in
+// fp32.  CTA (bh, column block of 32) computes out[:, 32 cb ..]; thread (ty,
+// tx) four rows x four columns, the reduction over 128 in slabs of 32.
+__global__ void __launch_bounds__(256) affine_step_kernel(const float *__restrict__ SI, const float *__restrict__ SZ,
+                                                          const float *__restrict__ X, float *__restrict__ out) {
+    __shared__ float Ms[DK][33];
+    __shared__ __align__(16) float Xs[32][36];
+    const size_t base = (size_t)blockIdx.x * DK * DK;
+    const int cb = 32 * blockIdx.y, tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < DK; k0 += 32) {
+        for (int e = tid; e < DK * 32; e += 256) {
+            const int r = e >> 5, c = e & 31;
+            const size_t a = base + (size_t)r * DK + k0 + c;
+            Ms[r][c] = SI[a] - SZ[a];
+        }
+        for (int e = tid; e < 32 * 32; e += 256) {
+            const int r = e >> 5, c = e & 31;
+            Xs[r][c] = X[base + (size_t)(k0 + r) * DK + cb + c];
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+            const float4 b = *reinterpret_cast<const float4 *>(&Xs[k][4 * tx]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float a = Ms[4 * ty + i][k];
+                acc[i][0] = fmaf(a, b.x, acc[i][0]);
+                acc[i][1] = fmaf(a, b.y, acc[i][1]);
+                acc[i][2] = fmaf(a, b.z, acc[i][2]);
+                acc[i][3] = fmaf(a, b.w, acc[i][3]);
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const size_t a = base + (size_t)(4 * ty + i) * DK + cb + 4 * tx + j;
+            out[a] = acc[i][j] + SZ[a];
+        }
+}
 
 template <typename Tout>
 inline efla_status_t launch(const void *q, const void *k, const void *v, const float *beta, const float *S0,
@@ -1012,8 +1119,43 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     chunk_prep_tc_kernel<<<(unsigned)(bh * nc), kPrepThreads, P_SMEM, st>>>(mq, mk, mv, beta, img, L, nc,
                                                                             euler ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
-    chunk_tc_kernel<Tout><<<(unsigned)grid, kThreads, SMEM_BYTES, st>>>(mq, mk, mo, img, S0, SL, L, nc);
-    return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
+    const int P = segments(bh, nc);
+    auto run = [&](const SegPlan &plan) {
+        chunk_tc_kernel<Tout><<<dim3((unsigned)grid, (unsigned)plan.njobs), kThreads, SMEM_BYTES, st>>>(mq, mk, mo,
+                                                                                                      img, plan);
+        return cudaGetLastError() == cudaSuccess;
+    };
+    SegPlan plan{};
+    plan.nc = nc;
+    if (P == 1) {
+        plan.njobs = 1;
+        plan.job[0] = SegJob{0, nc, S0 ? 1 : 0, 1, S0, SL};
+        return run(plan) ? EFLA_OK : EFLA_ERR_CUDA;
+    }
+    float *sbuf = reinterpret_cast<float *>(img + (size_t)bh * nc * PREP_BYTES);
+    const size_t sb = state_bytes(bh) / sizeof(float);
+    auto Sin = [&](int r) { return sbuf + (size_t)(r - 1) * sb; };               // r = 1 .. P-1
+    auto SZ = [&](int r) { return sbuf + (size_t)(P - 1 + r - 1) * sb; };         // r = 1 .. P-2
+    auto SI = [&](int r) { return sbuf + (size_t)(2 * P - 3 + r - 1) * sb; };     // r = 1 .. P-2
+    auto first = [&](int r) { return (int)((long)r * nc / P); };
+    // pass A
+    plan.njobs = 0;
+    plan.job[plan.njobs++] = SegJob{0, first(1), S0 ? 1 : 0, 1, S0, Sin(1)};
+    for (int r = 1; r <= P - 2; ++r) {
+        plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 0, 0, nullptr, SZ(r)};
+        plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 2, 0, nullptr, SI(r)};
+    }
+    if (!run(plan)) return EFLA_ERR_CUDA;
+    // the segment chain
+    for (int r = 1; r <= P - 2; ++r) {
+        affine_step_kernel<<<dim3((unsigned)bh, DK / 32), 256, 0, st>>>(SI(r), SZ(r), Sin(r), Sin(r + 1));
+        if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
+    }
+    // pass B
+    plan.njobs = 0;
+    for (int r = 1; r <= P - 1; ++r)
+        plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 1, 1, Sin(r), r == P - 1 ? SL : nullptr};
+    return run(plan) ? EFLA_OK : EFLA_ERR_CUDA;
 }
 
 }  // namespace tc

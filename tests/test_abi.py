@@ -96,3 +96,20 @@ def test_workspace_size_is_pure_and_scales(lib):
     assert so.efla_chunk_fwd_workspace_size(0, 4, 16, 8192, 128, 128) == 2 * a
     assert so.efla_chunk_fwd_workspace_size(0, 2, 16, 8192, 48, 48) == 0
     assert so.efla_chunk_fwd_workspace_size(0, 0, 16, 8192, 128, 128) == 0
+
+
+def test_bf16_workspace_includes_segment_states(lib):
+    # bf16 d=128 path: one 56 KB image per (b, h, chunk); with too few heads to
+    # fill the GPU the prefill is segmented (P segments) and adds 3P - 5 fp32
+    # states of d x d per (b, h).  Without a GPU the plan assumes 148 SMs.
+    so, _ = lib
+    img = 7 * 8192
+    st = 128 * 128 * 4
+    # 64 heads, 32 chunks: a single pass
+    assert so.efla_chunk_fwd_workspace_size(1, 8, 8, 2048, 128, 128) == 64 * 32 * img
+    # 16 heads, 1024 chunks: P = 3 (pass A needs 2 * 16 * 3 = 96 CTAs)
+    assert so.efla_chunk_fwd_workspace_size(1, 1, 16, 65536, 128, 128) == 16 * 1024 * img + 4 * 16 * st
+    # 2 heads, 128 chunks: P = 8 (16 chunks per segment)
+    assert so.efla_chunk_fwd_workspace_size(1, 1, 2, 8192, 128, 128) == 2 * 128 * img + 19 * 2 * st
+    # too few chunks per segment: a single pass
+    assert so.efla_chunk_fwd_workspace_size(1, 1, 2, 2048, 128, 128) == 2 * 32 * img
