@@ -328,6 +328,8 @@ def run_ours(args):
 
     if rank == 0 and not args.no_decode:
         line["decode"] = bench_decode(efla, dev, args, peaks)
+    if rank == 0 and not args.no_longctx:
+        line["longctx_prefill"] = bench_longctx(efla, dev, peaks)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(efla, dev, x, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -346,6 +348,39 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def bench_longctx(efla, dev, peaks, calls=10):
+    """The long-context prefill (B=1, H=16, L=65536, bf16 q/k/v, fp32 o and
+    state): 16 heads leave most SMs idle, so the library runs it
+    segment-parallel.  Same input twice (1.1 GB of inputs and outputs,
+    > L2), CUDA events over `calls` calls after 3 warm-up calls."""
+    x = workloads.chunk_inputs("longctx")
+    q, k, v, beta = (x[n].to(dev) for n in ("q", "k", "v", "beta"))
+    B, H, L, d = k.shape
+    o = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
+    S = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(efla.workspace_size(q.dtype, B, H, L, d, d), dtype=torch.uint8, device=dev)
+    call = lambda: efla.chunk_fwd(q, k, v, beta, None, o=o, S_L=S, workspace=ws)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(calls):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    if efla.last_error() != 0:
+        raise RuntimeError("efla_chunk_fwd reported a device-side error")
+    ms = e0.elapsed_time(e1) / calls
+    nbytes = chunk_bytes(B, H, L, d, 2, 4, s0=False)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"value": B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms, "calls": calls,
+            "config": f"longctx prefill: B={B} H={H} L={L} d={d} C=64 bf16 q/k/v, fp32 o/state, S0=0",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm"], "traffic": None, "kernel": "efla_chunk_fwd (all launches)",
+                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"]}}
 
 
 def bench_decode(efla, dev, args, peaks):
@@ -436,6 +471,7 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-longctx", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
