@@ -41,7 +41,8 @@ STATUS = {0: "EFLA_OK", 1: "EFLA_ERR_NULL", 2: "EFLA_ERR_SHAPE", 3: "EFLA_ERR_DT
           9: "EFLA_ERR_ALIAS"}
 EXPORTS = ("efla_status_string", "efla_version", "efla_last_error", "efla_gate",
            "efla_chunk_fwd_workspace_size", "efla_chunk_fwd", "efla_decode_step",
-           "efla_chunk_fwd_workspace_size_simt", "efla_chunk_fwd_noalloc", "efla_diag_wait_timeout")
+           "efla_chunk_fwd_workspace_size_simt", "efla_chunk_fwd_noalloc", "efla_diag_wait_timeout",
+           "efla_state_affine")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _p, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -65,6 +66,8 @@ _lib.efla_diag_wait_timeout.restype = _i
 _lib.efla_diag_wait_timeout.argtypes = [ctypes.c_longlong, _p]
 _lib.efla_decode_step.restype = _i
 _lib.efla_decode_step.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+_lib.efla_state_affine.restype = _i
+_lib.efla_state_affine.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
 
 
 class EflaError(RuntimeError):
@@ -219,3 +222,23 @@ def decode_step(q, k, v, beta, S, mode: str = "exact", o=None, out_dtype=torch.f
         _check(_lib.efla_decode_step(_ptr(q), _ptr(k), _ptr(v), _dt(q), MODES[mode], _ptr(beta), _ptr(S),
                                      _ptr(o), _dt(o), B, H, dk, dv, _stream(dev)), "efla_decode_step")
     return o
+
+
+def state_affine(SI, SZ, X, out=None):
+    """(SI - SZ) @ X + SZ for every (b, h): [B,H,d,d] fp32, d in {32, 64, 128}.
+    With SI / SZ the final states of a segment from the identity / from zero
+    and X the segment's true initial state, the result is its true final
+    state (the state map of a segment is affine)."""
+    dev = _dev(SI, SZ, X, out)
+    for t in (SI, SZ, X):
+        if t.dtype != torch.float32 or t.dim() != 4 or t.shape != SI.shape or not t.is_contiguous():
+            raise ValueError("SI, SZ, X must be contiguous float32 [B,H,d,d] of one shape")
+    B, H, d, d2 = SI.shape
+    if d != d2:
+        raise ValueError("square states only")
+    if out is None:
+        out = torch.empty_like(SI)
+    _check(_lib.efla_state_affine(_ptr(SI), _ptr(SZ), _ptr(X), _ptr(out), B, H, d, _stream(dev)),
+           "efla_state_affine")
+    return out
+

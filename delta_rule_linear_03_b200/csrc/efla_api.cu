@@ -293,6 +293,27 @@ efla_status_t efla_decode_step(const void *q, const void *k, const void *v, efla
     EFLA_DISPATCH(launch_decode, dtype, o_dtype, d_k, q, k, v, beta, S, o, bh, eu, st);
 }
 
+efla_status_t efla_state_affine(const float *SI, const float *SZ, const float *X, float *out, int B, int H, int d,
+                                efla_stream_t stream) {
+    if (B < 0 || H < 0) return EFLA_ERR_SHAPE;
+    if (d != 32 && d != 64 && d != 128) return EFLA_ERR_UNSUPPORTED;
+    const long long bh = (long long)B * H;
+    if (bh * d * d > kMaxElems || bh > 0x7fffffffLL) return EFLA_ERR_SHAPE;
+    if (bh == 0) return EFLA_OK;
+    if (!SI || !SZ || !X || !out) return EFLA_ERR_NULL;
+    if (!aligned16(SI) || !aligned16(SZ) || !aligned16(X) || !aligned16(out)) return EFLA_ERR_ALIGN;
+    const size_t sb = (size_t)bh * d * d * sizeof(float);
+    if (overlaps(out, sb, SI, sb) || overlaps(out, sb, SZ, sb) || overlaps(out, sb, X, sb)) return EFLA_ERR_ALIAS;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)bh, (unsigned)(d / 32));
+    switch (d) {
+        case 32: tc::affine_step_kernel<32><<<grid, 256, 0, st>>>(SI, SZ, X, out); break;
+        case 64: tc::affine_step_kernel<64><<<grid, 256, 0, st>>>(SI, SZ, X, out); break;
+        default: tc::affine_step_kernel<128><<<grid, 256, 0, st>>>(SI, SZ, X, out); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

@@ -1055,46 +1055,52 @@ inline size_t workspace_bytes(long bh, int L) {
     return (size_t)bh * nc * PREP_BYTES + (P > 1 ? (size_t)(3 * P - 5) * state_bytes(bh) : 0);
 }
 
-// out = (SI - SZ) X + SZ for every (b, h): one step of the segment chain, in
-// fp32.  CTA (bh, column block of 32) computes out[:, 32 cb ..]; thread (ty,
-// tx) four rows x four columns, the reduction over 128 in slabs of 32.
+// out = (SI - SZ) X + SZ for every (b, h), D x D fp32 matrices: one step of
+// the segment chain.  CTA (bh, column block of 32) computes out[:, 32 cb ..];
+// thread (ty, tx) four rows x four columns, the reduction in slabs of 32.
+template <int D>
 __global__ void __launch_bounds__(256) affine_step_kernel(const float *__restrict__ SI, const float *__restrict__ SZ,
                                                           const float *__restrict__ X, float *__restrict__ out) {
-    __shared__ float Ms[DK][33];
+    static_assert(D % 32 == 0 && D <= 128, "D in {32, 64, 128}");
+    __shared__ float Ms[D][33];
     __shared__ __align__(16) float Xs[32][36];
-    const size_t base = (size_t)blockIdx.x * DK * DK;
+    const size_t base = (size_t)blockIdx.x * D * D;
     const int cb = 32 * blockIdx.y, tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
+    const bool active = 4 * ty < D;
     float acc[4][4] = {};
-    for (int k0 = 0; k0 < DK; k0 += 32) {
-        for (int e = tid; e < DK * 32; e += 256) {
+    for (int k0 = 0; k0 < D; k0 += 32) {
+        for (int e = tid; e < D * 32; e += 256) {
             const int r = e >> 5, c = e & 31;
-            const size_t a = base + (size_t)r * DK + k0 + c;
+            const size_t a = base + (size_t)r * D + k0 + c;
             Ms[r][c] = SI[a] - SZ[a];
         }
         for (int e = tid; e < 32 * 32; e += 256) {
             const int r = e >> 5, c = e & 31;
-            Xs[r][c] = X[base + (size_t)(k0 + r) * DK + cb + c];
+            Xs[r][c] = X[base + (size_t)(k0 + r) * D + cb + c];
         }
         __syncthreads();
+        if (active) {
 #pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-            const float4 b = *reinterpret_cast<const float4 *>(&Xs[k][4 * tx]);
+            for (int k = 0; k < 32; ++k) {
+                const float4 b = *reinterpret_cast<const float4 *>(&Xs[k][4 * tx]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float a = Ms[4 * ty + i][k];
-                acc[i][0] = fmaf(a, b.x, acc[i][0]);
-                acc[i][1] = fmaf(a, b.y, acc[i][1]);
-                acc[i][2] = fmaf(a, b.z, acc[i][2]);
-                acc[i][3] = fmaf(a, b.w, acc[i][3]);
+                for (int i = 0; i < 4; ++i) {
+                    const float a = Ms[4 * ty + i][k];
+                    acc[i][0] = fmaf(a, b.x, acc[i][0]);
+                    acc[i][1] = fmaf(a, b.y, acc[i][1]);
+                    acc[i][2] = fmaf(a, b.z, acc[i][2]);
+                    acc[i][3] = fmaf(a, b.w, acc[i][3]);
+                }
             }
         }
         __syncthreads();
     }
+    if (!active) return;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const size_t a = base + (size_t)(4 * ty + i) * DK + cb + 4 * tx + j;
+            const size_t a = base + (size_t)(4 * ty + i) * D + cb + 4 * tx + j;
             out[a] = acc[i][j] + SZ[a];
         }
 }
@@ -1148,7 +1154,7 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     if (!run(plan)) return EFLA_ERR_CUDA;
     // the segment chain
     for (int r = 1; r <= P - 2; ++r) {
-        affine_step_kernel<<<dim3((unsigned)bh, DK / 32), 256, 0, st>>>(SI(r), SZ(r), Sin(r), Sin(r + 1));
+        affine_step_kernel<DK><<<dim3((unsigned)bh, DK / 32), 256, 0, st>>>(SI(r), SZ(r), Sin(r), Sin(r + 1));
         if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
     }
     // pass B

@@ -167,6 +167,23 @@ efla_status_t efla_decode_step(const void *q, const void *k, const void *v,
                                int d_v, efla_stream_t stream);
 
 /*
+ * efla_state_affine - one step of composing the state maps of consecutive
+ * sequence segments: for every (b, h),
+ *     out = (SI - SZ) X + SZ
+ * The state after a segment is affine in the state before it (the
+ * recurrence of 关键设计 2 is linear in S): S_out = M S_in + S_Z, where
+ * S_Z is the final state from S_in = 0, S_I the final state from the
+ * identity and M = S_I - S_Z.  With SI = S_I, SZ = S_Z and X a segment's
+ * true initial state, `out` is the next segment's true initial state.  The
+ * pages have no such call; sequence-parallel prefill (across GPUs or SMs)
+ * is built on it.
+ *   SI, SZ, X, out [B][H][d][d] fp32, d = d_k = d_v in {32, 64, 128}.
+ *   out must not overlap SI, SZ or X.  Asynchronous on `stream`.
+ */
+efla_status_t efla_state_affine(const float *SI, const float *SZ, const float *X, float *out,
+                                int B, int H, int d, efla_stream_t stream);
+
+/*
  * efla_chunk_fwd_noalloc - the same prefill as efla_chunk_fwd, for callers
  * that cannot allocate device memory.  The pages describe no such call; it
  * exists for this library's users.  Some hosts (inference engines and

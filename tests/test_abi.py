@@ -113,3 +113,16 @@ def test_bf16_workspace_includes_segment_states(lib):
     assert so.efla_chunk_fwd_workspace_size(1, 1, 2, 8192, 128, 128) == 2 * 128 * img + 19 * 2 * st
     # too few chunks per segment: a single pass
     assert so.efla_chunk_fwd_workspace_size(1, 1, 2, 2048, 128, 128) == 2 * 32 * img
+
+
+def test_state_affine_validation(lib):
+    import ctypes
+    so, _ = lib
+    p = ctypes.c_void_p(16)
+    so.efla_state_affine.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 3 + [ctypes.c_void_p]
+    assert so.efla_state_affine(p, p, p, ctypes.c_void_p(1 << 20), 1, 1, 48, None) == 5  # UNSUPPORTED
+    assert so.efla_state_affine(None, p, p, p, 1, 1, 64, None) == 1                      # NULL
+    assert so.efla_state_affine(p, p, p, p, -1, 1, 64, None) == 2                        # SHAPE
+    assert so.efla_state_affine(p, p, p, p, 0, 1, 64, None) == 0                         # empty: OK
+    assert so.efla_state_affine(p, p, p, ctypes.c_void_p(20), 1, 1, 64, None) == 4       # ALIGN
+    assert so.efla_state_affine(p, p, p, p, 1, 1, 64, None) == 9                         # ALIAS

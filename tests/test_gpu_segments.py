@@ -67,3 +67,46 @@ def test_segmented_in_place_state(efla):
     assert efla.last_error() == 0
     _, rS = oracle.recurrence(x["q"], x["k"], x["v"], x["beta"], x["S0"])
     assert_close(S, rS, "bf16", "S_L in place")
+
+
+def test_state_affine_matches_fp64(efla):
+    g = torch.Generator().manual_seed(3)
+    for d in (32, 64, 128):
+        SI, SZ, X = (torch.randn(2, 3, d, d, generator=g) for _ in range(3))
+        out = efla.state_affine(SI.cuda(), SZ.cuda(), X.cuda())
+        torch.cuda.synchronize()
+        ref = torch.matmul(SI.double() - SZ.double(), X.double()) + SZ.double()
+        err = (out.cpu().double() - ref).abs().max().item() / ref.abs().max().item()
+        assert err < 1e-5, f"d={d}: rel err {err:.2e}"
+
+
+def test_sequence_sharded_helper_on_one_gpu(efla):
+    # the rank-by-rank steps of the sequence-sharded helper, run here one
+    # segment after another on one GPU with the library's kernels
+    from delta_rule_linear_03_b200.sequence_parallel import initial_state
+    x = workloads.chunk_inputs("lm1p3b", B=1, H=2, L=700)
+    S0 = x["S0"].cuda()
+    bounds = [(0, 200), (200, 457), (457, 700)]
+    d = 128
+    eye = torch.eye(d, device="cuda").expand(1, 2, d, d).contiguous()
+    zero = torch.zeros(1, 2, d, d, device="cuda")
+    segs = [{n: x[n][:, :, a:b].contiguous().cuda() for n in ("q", "k", "v", "beta")} for a, b in bounds]
+    maps = []
+    for r, s in enumerate(segs):
+        if r == 0:
+            _, S_end = efla.chunk_fwd(s["q"], s["k"], s["v"], s["beta"], S0)
+            maps.append((S_end, S_end))
+        else:
+            _, SZ = efla.chunk_fwd(s["q"], s["k"], s["v"], s["beta"], zero)
+            _, SI = efla.chunk_fwd(s["q"], s["k"], s["v"], s["beta"], eye)
+            maps.append((SZ, SI))
+    outs = []
+    for r, s in enumerate(segs):
+        S_in = initial_state(maps, S0, r, efla.state_affine)
+        o, S_last = efla.chunk_fwd(s["q"], s["k"], s["v"], s["beta"], S_in.contiguous())
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert efla.last_error() == 0
+    ro, rS = oracle.recurrence(x["q"], x["k"], x["v"], x["beta"], x["S0"])
+    assert_close(torch.cat(outs, dim=2), ro, "bf16", "o")
+    assert_close(S_last, rS, "bf16", "S_L")
