@@ -76,6 +76,8 @@ def _load():
         lib.efla_oracle_recurrence.argtypes = [p, p, p, p, p, i, i, i, i, i, i, p, p, i]
         lib.efla_oracle_chunked.restype = None
         lib.efla_oracle_chunked.argtypes = [p, p, p, p, p, i, i, i, i, i, i, i, p, p, i]
+        lib.efla_oracle_backward.restype = None
+        lib.efla_oracle_backward.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, p, p, p, p, p, i]
         lib.efla_oracle_expm_taylor.restype = None
         lib.efla_oracle_expm_taylor.argtypes = [i, p, d, p]
         lib.efla_oracle_duhamel.restype = None
@@ -142,6 +144,24 @@ def recurrence(q, k, v, beta, S0=None, euler: bool = False, threads: int | None 
         B, H, L, dk, dv, int(euler), _ptr(o) if o is not None else None, _ptr(SL),
         threads or default_threads())
     return o, SL
+
+
+def backward(q, k, v, beta, S0, dO, dSL=None, euler: bool = False, threads: int | None = None):
+    """Reverse-mode derivative of ``recurrence`` for the loss
+    L = sum(dO * o) + sum(dSL * S_L): returns (dq, dk, dv, dbeta, dS0) in fp64."""
+    q, k, v, beta, S0, B, H, L, dk, dv = _prep(q, k, v, beta, S0)
+    dO = _f64(dO)
+    assert dO.shape == (B, H, L, dv)
+    if dSL is not None:
+        dSL = _f64(dSL)
+        assert dSL.shape == (B, H, dk, dv)
+    dq, dkk = np.empty((B, H, L, dk)), np.empty((B, H, L, dk))
+    dvv, dbeta, dS0 = np.empty((B, H, L, dv)), np.empty((B, H, L)), np.empty((B, H, dk, dv))
+    _load().efla_oracle_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(S0) if S0 is not None else None, _ptr(dO),
+        _ptr(dSL) if dSL is not None else None, B, H, L, dk, dv, int(euler),
+        _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dbeta), _ptr(dS0), threads or default_threads())
+    return dq, dkk, dvv, dbeta, dS0
 
 
 def chunked(q, k, v, beta, S0=None, C: int = 64, euler: bool = False,

@@ -103,6 +103,125 @@ void efla_oracle_recurrence(const double *q, const double *k, const double *v,
     }
 }
 
+/* Derivatives of the gate alpha(beta, lambda) of efla_oracle_alpha: with
+ * x = beta * lambda, d alpha / d beta = e^{-x} and
+ *     d alpha / d lambda = (x e^{-x} - (1 - e^{-x})) / lambda^2,
+ * summed as its series beta^2 * sum_{n>=2} (-1)^{n+1} (n-1) x^{n-2} / n!
+ * for |x| < 1e-3 (the closed form cancels there).  Where the clamp
+ * lambda <= 1e-12 is active alpha does not depend on lambda.  Euler: alpha =
+ * beta. */
+static void alpha_grad(double beta, double lambda, int euler, double *da_db, double *da_dl)
+{
+    if (euler) { *da_db = 1.0; *da_dl = 0.0; return; }
+    if (lambda <= EFLA_ORACLE_EPS) {
+        *da_db = exp(-beta * EFLA_ORACLE_EPS);
+        *da_dl = 0.0;
+        return;
+    }
+    double x = beta * lambda;
+    *da_db = exp(-x);
+    if (fabs(x) < 1e-3) {
+        double sum = 0.0, xp = 1.0, fact = 2.0;  /* n = 2: x^0 / 2! */
+        for (int n = 2; n < 10; ++n) {
+            double term = (double)(n - 1) * xp / fact;
+            sum += (n % 2 == 1) ? term : -term;  /* (-1)^{n+1} */
+            xp *= x;
+            fact *= (double)(n + 1);
+        }
+        *da_dl = beta * beta * sum;
+    } else {
+        *da_dl = (x * exp(-x) + expm1(-x)) / (lambda * lambda);
+    }
+}
+
+/* Reverse-mode derivative of the sequential recurrence, for every (b,h),
+ * given dO = dL/do [B,H,L,dv] and dSL = dL/dS_L [B,H,dk,dv] (NULL = 0).
+ * The forward states S_0..S_L are kept in full.  Backwards over t, with
+ * H = dL/dS_t (the readout of step t included, H += q_t do_t^T):
+ *   e = v_t - S_{t-1}^T k_t,  g = H^T k_t,
+ *   d alpha = g . e,          de = alpha g        (= dv_t)
+ *   dq_t = S_t do_t,          dk_t = alpha H e - S_{t-1} de
+ *                                    + 2 d alpha (d alpha/d lambda) k_t
+ *   dbeta_t = d alpha (d alpha/d beta)
+ *   H <- H - k_t de^T         (= (I - alpha k_t k_t^T) H)
+ * and dS0 = H at the end.  Outputs: dq, dk [B,H,L,dk], dv [B,H,L,dv],
+ * dbeta [B,H,L], dS0 [B,H,dk,dv]. */
+void efla_oracle_backward(const double *q, const double *k, const double *v,
+                          const double *beta, const double *S0, const double *dO,
+                          const double *dSL, int B, int H, int L, int dk, int dv,
+                          int euler, double *dq, double *dkk, double *dvv,
+                          double *dbeta, double *dS0, int nthreads)
+{
+    long BH = (long)B * H;
+    long SS = (long)dk * dv;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads > 0 ? nthreads : 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        double *S = (double *)malloc(sizeof(double) * (size_t)(L + 1) * SS);
+        double *Hm = (double *)malloc(sizeof(double) * (size_t)SS);
+        double *kts = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *e = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *g = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *de = (double *)malloc(sizeof(double) * (size_t)dv);
+        if (S0) memcpy(S, S0 + bh * SS, sizeof(double) * (size_t)SS);
+        else memset(S, 0, sizeof(double) * (size_t)SS);
+        for (int t = 0; t < L; ++t) {
+            long row = bh * L + t;
+            const double *kt = k + row * dk;
+            double lam = 0.0;
+            for (int i = 0; i < dk; ++i) lam += kt[i] * kt[i];
+            double a = efla_oracle_alpha(beta[row], lam, euler);
+            memcpy(S + (long)(t + 1) * SS, S + (long)t * SS, sizeof(double) * (size_t)SS);
+            one_token(dk, dv, q + row * dk, kt, v + row * dv, a, S + (long)(t + 1) * SS, NULL, kts);
+        }
+        if (dSL) memcpy(Hm, dSL + bh * SS, sizeof(double) * (size_t)SS);
+        else memset(Hm, 0, sizeof(double) * (size_t)SS);
+        for (int t = L - 1; t >= 0; --t) {
+            long row = bh * L + t;
+            const double *qt = q + row * dk, *kt = k + row * dk, *vt = v + row * dv, *dot = dO + row * dv;
+            const double *Sp = S + (long)t * SS, *Sn = S + (long)(t + 1) * SS;
+            double lam = 0.0;
+            for (int i = 0; i < dk; ++i) lam += kt[i] * kt[i];
+            double a = efla_oracle_alpha(beta[row], lam, euler), da_db, da_dl;
+            alpha_grad(beta[row], lam, euler, &da_db, &da_dl);
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) Hm[(long)i * dv + j] += qt[i] * dot[j];
+            for (int i = 0; i < dk; ++i) {  /* dq_t = S_t do_t */
+                double acc = 0.0;
+                for (int j = 0; j < dv; ++j) acc += Sn[(long)i * dv + j] * dot[j];
+                dq[row * dk + i] = acc;
+            }
+            for (int j = 0; j < dv; ++j) {
+                double se = 0.0, hg = 0.0;
+                for (int i = 0; i < dk; ++i) {
+                    se += Sp[(long)i * dv + j] * kt[i];
+                    hg += Hm[(long)i * dv + j] * kt[i];
+                }
+                e[j] = vt[j] - se;
+                g[j] = hg;
+            }
+            double dal = 0.0;
+            for (int j = 0; j < dv; ++j) dal += g[j] * e[j];
+            for (int j = 0; j < dv; ++j) {
+                de[j] = a * g[j];
+                dvv[row * dv + j] = de[j];
+            }
+            for (int i = 0; i < dk; ++i) {
+                double he = 0.0, sde = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    he += Hm[(long)i * dv + j] * e[j];
+                    sde += Sp[(long)i * dv + j] * de[j];
+                }
+                dkk[row * dk + i] = a * he - sde + 2.0 * dal * da_dl * kt[i];
+            }
+            dbeta[row] = dal * da_db;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) Hm[(long)i * dv + j] -= kt[i] * de[j];
+        }
+        memcpy(dS0 + bh * SS, Hm, sizeof(double) * (size_t)SS);
+        free(S); free(Hm); free(kts); free(e); free(g); free(de);
+    }
+}
+
 /* Chunked (UT-form) evaluation of the same recurrence, in fp64, written
  * independently of the sequential loop above.  It is the scheme the pages
  * cite for training (整体框架: chunks of size C, tensorised products) and is
