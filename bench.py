@@ -330,6 +330,8 @@ def run_ours(args):
         line["decode"] = bench_decode(efla, dev, args, peaks)
     if rank == 0 and not args.no_longctx:
         line["longctx_prefill"] = bench_longctx(efla, dev, peaks)
+    if rank == 0 and not args.no_backward:
+        line["backward"] = bench_backward(efla, dev, x, peaks)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(efla, dev, x, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -348,6 +350,34 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def bench_backward(efla, dev, x, peaks, calls=5):
+    """efla_prefill_bwd on the timed workload (one fp32 dO, no S0/dS_L):
+    exact fp32, one CTA per (b, h) walking the sequence three times."""
+    q, k, v, beta = (x[n].to(dev) for n in ("q", "k", "v", "beta"))
+    B, H, L, d = k.shape
+    dO = torch.randn(B, H, L, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+    ws = torch.empty(efla.prefill_bwd_workspace_size(B, H, L, d), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        efla.prefill_bwd(q, k, v, beta, None, dO, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(calls):
+        efla.prefill_bwd(q, k, v, beta, None, dO, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    if efla.last_error() != 0:
+        raise RuntimeError("efla_prefill_bwd reported a device-side error")
+    ms = e0.elapsed_time(e1) / calls
+    # HBM bytes: read q, k, v, beta, dO (x2 passes for k); write dq, dk, dv, dbeta; e_t round trip
+    tok = B * H * L
+    nbytes = tok * (3 * d * 2 + 4 + d * 4 + 3 * d * 4 + 4 + 2 * d * 4)
+    return {"value": B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms, "calls": calls,
+            "config": f"{WORKLOAD} backward: dq, dk, dv, dbeta, dS0 (fp32), bf16 q/k/v, fp32 dO",
+            "kernel": "backward_kernel (fp32, serial over tokens per (b, h))",
+            "hbm_bytes_estimate": nbytes}
 
 
 def bench_longctx(efla, dev, peaks, calls=10):
@@ -472,6 +502,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-longctx", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

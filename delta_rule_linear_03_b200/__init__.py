@@ -42,7 +42,7 @@ STATUS = {0: "EFLA_OK", 1: "EFLA_ERR_NULL", 2: "EFLA_ERR_SHAPE", 3: "EFLA_ERR_DT
 EXPORTS = ("efla_status_string", "efla_version", "efla_last_error", "efla_gate",
            "efla_chunk_fwd_workspace_size", "efla_chunk_fwd", "efla_decode_step",
            "efla_chunk_fwd_workspace_size_simt", "efla_chunk_fwd_noalloc", "efla_diag_wait_timeout",
-           "efla_state_affine")
+           "efla_state_affine", "efla_prefill_bwd_workspace_size", "efla_prefill_bwd")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _p, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -68,6 +68,11 @@ _lib.efla_decode_step.restype = _i
 _lib.efla_decode_step.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.efla_state_affine.restype = _i
 _lib.efla_state_affine.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
+_lib.efla_prefill_bwd_workspace_size.restype = _sz
+_lib.efla_prefill_bwd_workspace_size.argtypes = [_i, _i, _i, _i, _i]
+_lib.efla_prefill_bwd.restype = _i
+_lib.efla_prefill_bwd.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                                  _i, _i, _i, _i, _i, _p, _sz, _p]
 
 
 class EflaError(RuntimeError):
@@ -239,6 +244,41 @@ def state_affine(SI, SZ, X, out=None):
     if out is None:
         out = torch.empty_like(SI)
     _check(_lib.efla_state_affine(_ptr(SI), _ptr(SZ), _ptr(X), _ptr(out), B, H, d, _stream(dev)),
-           "efla_state_affine")
+           "efla_state_affine", "efla_prefill_bwd_workspace_size", "efla_prefill_bwd")
     return out
+
+
+def prefill_bwd(q, k, v, beta, S0, dO, dSL=None, mode: str = "exact", workspace=None):
+    """Gradients of L = sum(dO * o) + sum(dSL * S_L) for ``chunk_fwd(q, k, v,
+    beta, S0)``: returns (dq, dk, dv [B,H,L,d], dbeta [B,H,L], dS0 [B,H,d,d]),
+    all float32.  q, k, v share one dtype (fp32 or bf16); beta, S0 (or
+    None), dO and dSL (or None) are float32."""
+    dev = _dev(q, k, v, beta, S0, dO, dSL)
+    B, H, L, dk_ = k.shape
+    dv_ = v.shape[-1]
+    if q.shape != k.shape or v.shape[:3] != (B, H, L) or q.dtype != k.dtype or v.dtype != k.dtype:
+        raise ValueError("q, k, v must share dtype and [B,H,L,*] shape")
+    for name, t, shape in (("beta", beta, (B, H, L)), ("dO", dO, (B, H, L, dv_)),
+                           ("S0", S0, (B, H, dk_, dv_)), ("dSL", dSL, (B, H, dk_, dv_))):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous()):
+            raise ValueError(f"{name} must be contiguous float32 {shape}")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    f = dict(dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty(B, H, L, dk_, **f), torch.empty(B, H, L, dk_, **f), torch.empty(B, H, L, dv_, **f)
+    dbeta, dS0 = torch.empty(B, H, L, **f), torch.empty(B, H, dk_, dv_, **f)
+    need = int(_lib.efla_prefill_bwd_workspace_size(B, H, L, dk_, dv_))
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.efla_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _dt(k), MODES[mode], _ptr(beta), _ptr(S0), _ptr(dO),
+                                 _ptr(dSL), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dS0), B, H, L, dk_, dv_,
+                                 _ptr(workspace) if need else None, wbytes if need else 0, _stream(dev)),
+           "efla_prefill_bwd")
+    return dq, dk, dv, dbeta, dS0
+
+
+def prefill_bwd_workspace_size(B: int, H: int, L: int, d: int) -> int:
+    return int(_lib.efla_prefill_bwd_workspace_size(B, H, L, d, d))
 

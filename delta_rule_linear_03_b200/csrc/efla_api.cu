@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "../../include/efla.h"
+#include "efla_backward.cuh"
 #include "efla_chunk_simt.cuh"
 #include "efla_chunk_tc.cuh"
 #include "efla_common.cuh"
@@ -291,6 +292,84 @@ efla_status_t efla_decode_step(const void *q, const void *k, const void *v, efla
     const bool eu = mode == EFLA_MODE_EULER;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     EFLA_DISPATCH(launch_decode, dtype, o_dtype, d_k, q, k, v, beta, S, o, bh, eu, st);
+}
+
+size_t efla_prefill_bwd_workspace_size(int B, int H, int L, int d_k, int d_v) {
+    if (B <= 0 || H <= 0 || L <= 0 || check_head(d_k, d_v) != EFLA_OK) return 0;
+    return (size_t)B * H * L * ((size_t)d_v + 1) * sizeof(float);  // e_t per token, and one scalar
+}
+
+}  // extern "C"
+
+namespace {
+template <typename T, int D>
+efla_status_t launch_bwd(const void *q, const void *k, const void *v, const float *beta, const float *S0,
+                         const float *dO, const float *dSL, float *dq, float *dk, float *dv, float *dbeta, float *dS0,
+                         long bh, int L, bool eu, void *ws, cudaStream_t st) {
+    float *E = static_cast<float *>(ws);
+    float *Cg = E + (size_t)bh * L * D;
+    efla::backward_kernel<T, D, D><<<(unsigned)bh, 256, 0, st>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta, S0, dO, dSL, dq, dk, dv,
+        dbeta, dS0, E, Cg, L, eu);
+    return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+efla_status_t efla_prefill_bwd(const void *q, const void *k, const void *v, efla_dtype_t dtype, efla_mode_t mode,
+                               const float *beta, const float *S0, const float *dO, const float *dSL, float *dq,
+                               float *dk, float *dv, float *dbeta, float *dS0, int B, int H, int L, int d_k, int d_v,
+                               void *workspace, size_t workspace_bytes, efla_stream_t stream) {
+    efla_status_t s = check_common(dtype, mode);
+    if (s != EFLA_OK) return s;
+    if (B < 0 || H < 0 || L < 0) return EFLA_ERR_SHAPE;
+    if ((s = check_head(d_k, d_v)) != EFLA_OK) return s;
+    const long long bh = (long long)B * H;
+    if (bh * (long long)(L > 0 ? L : 1) * d_k > kMaxElems || bh > 0x7fffffffLL) return EFLA_ERR_SHAPE;
+    if (bh == 0) return EFLA_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t sbytes = (size_t)bh * d_k * d_v * sizeof(float);
+    if (L == 0) {  // no tokens (per-token buffers may be NULL): dS0 = dSL
+        if (!dS0) return EFLA_ERR_NULL;
+        if (!aligned16(dS0) || (dSL && !aligned16(dSL))) return EFLA_ERR_ALIGN;
+        if (dSL && overlaps(dS0, sbytes, dSL, sbytes)) return EFLA_ERR_ALIAS;
+        if (dSL) return cudaMemcpyAsync(dS0, dSL, sbytes, cudaMemcpyDeviceToDevice, st) == cudaSuccess ? EFLA_OK
+                                                                                                     : EFLA_ERR_CUDA;
+        return cudaMemsetAsync(dS0, 0, sbytes, st) == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
+    }
+    if (!q || !k || !v || !beta || !dO || !dq || !dk || !dv || !dbeta || !dS0) return EFLA_ERR_NULL;
+    const void *ins[] = {q, k, v, beta, S0, dO, dSL};
+    const void *outs[] = {dq, dk, dv, dbeta, dS0};
+    for (const void *p : ins)
+        if (p && !aligned16(p)) return EFLA_ERR_ALIGN;
+    for (const void *p : outs)
+        if (!aligned16(p)) return EFLA_ERR_ALIGN;
+    const size_t xb = (size_t)bh * L * d_k * esize(dtype), fb = (size_t)bh * L * d_k * sizeof(float);
+    const size_t bb = (size_t)bh * L * sizeof(float);
+    const size_t in_b[] = {xb, xb, xb, bb, sbytes, fb, sbytes};
+    const size_t out_b[] = {fb, fb, fb, bb, sbytes};
+    for (int i = 0; i < 5; ++i) {
+        for (int j = 0; j < 7; ++j)
+            if (ins[j] && overlaps(outs[i], out_b[i], ins[j], in_b[j])) return EFLA_ERR_ALIAS;
+        for (int j = 0; j < i; ++j)
+            if (overlaps(outs[i], out_b[i], outs[j], out_b[j])) return EFLA_ERR_ALIAS;
+    }
+    const size_t need = efla_prefill_bwd_workspace_size(B, H, L, d_k, d_v);
+    if (!workspace || workspace_bytes < need) return EFLA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return EFLA_ERR_ALIGN;
+    const bool eu = mode == EFLA_MODE_EULER;
+    const bool bf = dtype == EFLA_BF16;
+#define EFLA_BWD(T, D) return launch_bwd<T, D>(q, k, v, beta, S0, dO, dSL, dq, dk, dv, dbeta, dS0, bh, L, eu, workspace, st)
+    if (bf) {
+        if (d_k == 32) EFLA_BWD(__nv_bfloat16, 32);
+        if (d_k == 64) EFLA_BWD(__nv_bfloat16, 64);
+        EFLA_BWD(__nv_bfloat16, 128);
+    }
+    if (d_k == 32) EFLA_BWD(float, 32);
+    if (d_k == 64) EFLA_BWD(float, 64);
+    EFLA_BWD(float, 128);
+#undef EFLA_BWD
 }
 
 efla_status_t efla_state_affine(const float *SI, const float *SZ, const float *X, float *out, int B, int H, int d,

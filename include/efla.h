@@ -167,6 +167,32 @@ efla_status_t efla_decode_step(const void *q, const void *k, const void *v,
                                int d_v, efla_stream_t stream);
 
 /*
+ * efla_prefill_bwd - reverse-mode derivative of efla_chunk_fwd.  The pages
+ * train with this mixer but print no backward; it is derived from the
+ * recurrence of 关键设计 2 (S_t = S_{t-1} + alpha_t k_t e_t^T with
+ * e_t = v_t - S_{t-1}^T k_t, o_t = S_t^T q_t) and the gate of 关键设计 2 /
+ * 损失函数 (d alpha/d beta = e^{-beta lambda}, d alpha/d lambda =
+ * (beta lambda e^{-beta lambda} - (1 - e^{-beta lambda})) / lambda^2, zero
+ * where lambda <= 1e-12).  For the loss sum(dO * o) + sum(dSL * S_L) it
+ * returns the gradients with respect to every input:
+ *   q, k [B][H][L][d]  v [B][H][L][d]  dtype `dtype`    (forward inputs)
+ *   beta [B][H][L] fp32, S0 [B][H][d][d] fp32 or NULL (zero state)
+ *   dO [B][H][L][d] fp32; dSL [B][H][d][d] fp32 or NULL (zero)
+ *   dq, dk, dv [B][H][L][d] fp32; dbeta [B][H][L] fp32; dS0 [B][H][d][d] fp32
+ *   workspace / workspace_bytes: caller-owned device scratch of at least
+ *     efla_prefill_bwd_workspace_size(...) bytes.
+ * d = d_k = d_v in {32, 64, 128}.  Exact fp32 arithmetic, one CTA per (b,h)
+ * walking the sequence three times (forward, backward, forward).  Outputs
+ * must not overlap inputs or each other.  Asynchronous on `stream`.
+ */
+size_t efla_prefill_bwd_workspace_size(int B, int H, int L, int d_k, int d_v);
+efla_status_t efla_prefill_bwd(const void *q, const void *k, const void *v, efla_dtype_t dtype, efla_mode_t mode,
+                               const float *beta, const float *S0, const float *dO, const float *dSL,
+                               float *dq, float *dk, float *dv, float *dbeta, float *dS0,
+                               int B, int H, int L, int d_k, int d_v,
+                               void *workspace, size_t workspace_bytes, efla_stream_t stream);
+
+/*
  * efla_state_affine - one step of composing the state maps of consecutive
  * sequence segments: for every (b, h),
  *     out = (SI - SZ) X + SZ

@@ -126,3 +126,34 @@ def test_state_affine_validation(lib):
     assert so.efla_state_affine(p, p, p, p, 0, 1, 64, None) == 0                         # empty: OK
     assert so.efla_state_affine(p, p, p, ctypes.c_void_p(20), 1, 1, 64, None) == 4       # ALIGN
     assert so.efla_state_affine(p, p, p, p, 1, 1, 64, None) == 9                         # ALIAS
+
+
+def test_prefill_bwd_validation(lib):
+    import ctypes
+    so, _ = lib
+    P = ctypes.c_void_p
+    so.efla_prefill_bwd.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int] + [P] * 9 + [ctypes.c_int] * 5 + \
+        [P, ctypes.c_size_t, P]
+    so.efla_prefill_bwd_workspace_size.restype = ctypes.c_size_t
+    ptrs = [P(16 * (i + 1) << 20) for i in range(12)]  # distinct, aligned, far apart
+    q, k, v, beta, S0, dO, dSL, dq, dk, dv, db, dS = ptrs
+    ws = P(64 << 30)
+
+    def call(**kw):
+        a = dict(q=q, k=k, v=v, dt=0, mode=0, beta=beta, S0=S0, dO=dO, dSL=dSL, dq=dq, dk=dk, dv=dv, db=db,
+                 dS=dS, B=1, H=2, L=8, dk_=64, dv_=64, ws=ws, wsb=1 << 30)
+        a.update(kw)
+        return so.efla_prefill_bwd(a["q"], a["k"], a["v"], a["dt"], a["mode"], a["beta"], a["S0"], a["dO"],
+                                   a["dSL"], a["dq"], a["dk"], a["dv"], a["db"], a["dS"], a["B"], a["H"], a["L"],
+                                   a["dk_"], a["dv_"], a["ws"], a["wsb"], None)
+
+    assert call(dq=None) == 1                      # NULL
+    assert call(dk_=48, dv_=48) == 5               # UNSUPPORTED head size
+    assert call(dt=7) == 3                         # DTYPE
+    assert call(L=-1) == 2                         # SHAPE
+    assert call(dq=P((16 << 20) + 4)) == 4         # ALIGN
+    assert call(dq=q) == 9                         # ALIAS (output over an input)
+    assert call(ws=None) == 8                      # WORKSPACE missing
+    assert call(wsb=16) == 8                       # WORKSPACE too small
+    assert call(B=0) == 0                          # empty batch: nothing to do
+    assert so.efla_prefill_bwd_workspace_size(1, 2, 8, 64, 64) == 2 * 8 * (64 + 1) * 4
