@@ -244,7 +244,7 @@ def state_affine(SI, SZ, X, out=None):
     if out is None:
         out = torch.empty_like(SI)
     _check(_lib.efla_state_affine(_ptr(SI), _ptr(SZ), _ptr(X), _ptr(out), B, H, d, _stream(dev)),
-           "efla_state_affine", "efla_prefill_bwd_workspace_size", "efla_prefill_bwd")
+           "efla_state_affine")
     return out
 
 

@@ -169,9 +169,9 @@ void efla_oracle_backward(const double *q, const double *k, const double *v,
             const double *kt = k + row * dk;
             double lam = 0.0;
             for (int i = 0; i < dk; ++i) lam += kt[i] * kt[i];
-            double a = efla_oracle_alpha(beta[row], lam, euler);
+            const double at = efla_oracle_alpha(beta[row], lam, euler);
             memcpy(S + (long)(t + 1) * SS, S + (long)t * SS, sizeof(double) * (size_t)SS);
-            one_token(dk, dv, q + row * dk, kt, v + row * dv, a, S + (long)(t + 1) * SS, NULL, kts);
+            one_token(dk, dv, q + row * dk, kt, v + row * dv, at, S + (long)(t + 1) * SS, NULL, kts);
         }
         if (dSL) memcpy(Hm, dSL + bh * SS, sizeof(double) * (size_t)SS);
         else memset(Hm, 0, sizeof(double) * (size_t)SS);
