@@ -1,6 +1,7 @@
 // efla_api.cu - the C ABI declared in include/efla.h: validation, scratch
 // sizing and kernel dispatch.  Every step of the computation runs in the
 // kernels included below; this file only checks arguments and launches.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -296,7 +297,7 @@ efla_status_t efla_decode_step(const void *q, const void *k, const void *v, efla
 
 size_t efla_prefill_bwd_workspace_size(int B, int H, int L, int d_k, int d_v) {
     if (B <= 0 || H <= 0 || L <= 0 || check_head(d_k, d_v) != EFLA_OK) return 0;
-    return (size_t)B * H * L * ((size_t)d_v + 1) * sizeof(float);  // e_t per token, and one scalar
+    return (size_t)B * H * L * ((size_t)d_v + 1 + 4) * sizeof(float);  // e_t, one scalar, the gate (float4)
 }
 
 }  // extern "C"
@@ -306,11 +307,16 @@ template <typename T, int D>
 efla_status_t launch_bwd(const void *q, const void *k, const void *v, const float *beta, const float *S0,
                          const float *dO, const float *dSL, float *dq, float *dk, float *dv, float *dbeta, float *dS0,
                          long bh, int L, bool eu, void *ws, cudaStream_t st) {
-    float *E = static_cast<float *>(ws);
+    float4 *G = static_cast<float4 *>(ws);  // first: 16-byte aligned
+    float *E = reinterpret_cast<float *>(G + (size_t)bh * L);
     float *Cg = E + (size_t)bh * L * D;
+    const long rows = bh * L;
+    const unsigned gblocks = (unsigned)std::min<long>((rows + 7) / 8, 148L * 16);
+    efla::backward_gate_kernel<T, D><<<gblocks, 256, 0, st>>>(static_cast<const T *>(k), beta, G, rows, eu);
+    if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
     efla::backward_kernel<T, D, D><<<(unsigned)bh, 256, 0, st>>>(
-        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), beta, S0, dO, dSL, dq, dk, dv,
-        dbeta, dS0, E, Cg, L, eu);
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), G, S0, dO, dSL, dq, dk, dv,
+        dbeta, dS0, E, Cg, L);
     return cudaGetLastError() == cudaSuccess ? EFLA_OK : EFLA_ERR_CUDA;
 }
 }  // namespace

@@ -156,4 +156,4 @@ def test_prefill_bwd_validation(lib):
     assert call(ws=None) == 8                      # WORKSPACE missing
     assert call(wsb=16) == 8                       # WORKSPACE too small
     assert call(B=0) == 0                          # empty batch: nothing to do
-    assert so.efla_prefill_bwd_workspace_size(1, 2, 8, 64, 64) == 2 * 8 * (64 + 1) * 4
+    assert so.efla_prefill_bwd_workspace_size(1, 2, 8, 64, 64) == 2 * 8 * (64 + 5) * 4
