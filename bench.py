@@ -56,6 +56,15 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ algorithmic work
+# DRAM bytes (read + write) of one lm340m efla_chunk_fwd call, summed over its
+# two launches, from one ncu capture of the current kernels
+# (dram__bytes_read.sum + dram__bytes_write.sum; prep 101.25 + 61.9 MB,
+# serial state kernel 184.6 + 40.5 MB).  Well above the 172.5 MB of
+# algorithmic bytes: the prep kernel's per-chunk workspace image (-W, M, U)
+# is written and read back once.
+CHUNK_TRAFFIC_LM340M = 388.3e6
+
+
 def chunk_bytes(B, H, L, d, esize, esize_o, s0: bool, sl: bool = True):
     """Algorithmic HBM bytes of one efla_chunk_fwd: read q, k, v and beta,
     write o, read S0 (if given) and write S_L once."""
@@ -315,7 +324,8 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.lm340m distribution)",
         "config": workload_config(w, world),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": achieved_gbs / peaks["hbm"], "traffic": None,
+                     "frac": achieved_gbs / peaks["hbm"],
+                     "traffic": CHUNK_TRAFFIC_LM340M if (WORKLOAD == "lm340m" and launches_per_step == 2) else None,
                      "kernel": "efla_chunk_fwd (all launches of one call)" if launches_per_step > 1
                      else "efla_chunk_fwd fused kernel",
                      "algorithmic_bytes": nbytes, "peak_source": peaks["source"]},
@@ -332,6 +342,8 @@ def run_ours(args):
         line["longctx_prefill"] = bench_longctx(efla, dev, peaks)
     if rank == 0 and not args.no_backward:
         line["backward"] = bench_backward(efla, dev, x, peaks)
+    if rank == 0:
+        line["gate"] = bench_gate(efla, dev, peaks)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(efla, dev, x, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -350,6 +362,46 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def bench_gate(efla, dev, peaks, reps=50):
+    """efla_gate alone on the lm1p3b keys (4 x 16 x 4096 bf16 rows of 128;
+    67 MB of k, > L2 with 4 rotating copies): alpha and lambda per key.
+    CUDA graph of 4 calls over the 4 copies, timed with CUDA events."""
+    sets = []
+    for i in range(4):
+        xi = workloads.chunk_inputs("lm1p3b", seed=100 + i)
+        sets.append((xi["k"].to(dev), xi["beta"].to(dev)))
+    B, H, L, d = sets[0][0].shape
+    outs = [(torch.empty(B, H, L, device=dev), torch.empty(B, H, L, device=dev)) for _ in range(4)]
+
+    def block():
+        for (k, b), (a, lam) in zip(sets, outs):
+            efla.gate(k, b, alpha=a, lam=lam)
+
+    for _ in range(3):
+        block()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        block()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (4 * reps)
+    rows = B * H * L
+    nbytes = rows * (2 * d + 4 + 8)  # read k (bf16) and beta, write alpha and lambda
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"value": rows / (ms / 1e3), "unit": "keys/s", "ms_per_call": ms, "calls": 4 * reps,
+            "config": f"lm1p3b keys: {B}x{H}x{L} rows of d={d} bf16, 4 rotating copies (> L2)",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm"], "traffic": None, "kernel": "gate_kernel",
+                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"]}}
 
 
 def bench_backward(efla, dev, x, peaks, calls=5):
