@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(256) gate_kernel(const T *__restrict__ k, cons
 
     for (long base = warp * (RPW * UNROLL); base < rows; base += nwarp * (RPW * UNROLL)) {
         uint4 raw[UNROLL];
+        float bt[UNROLL];  // beta, loaded with the keys so its latency overlaps theirs
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
             const long r = base + (long)u * RPW + sub;
@@ -37,6 +38,7 @@ __global__ void __launch_bounds__(256) gate_kernel(const T *__restrict__ k, cons
                 raw[u] = __ldcs(reinterpret_cast<const uint4 *>(k + r * D) + gl);
             else
                 raw[u] = make_uint4(0u, 0u, 0u, 0u);
+            bt[u] = (gl == 0 && r < rows) ? __ldcs(beta + r) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
@@ -51,7 +53,7 @@ __global__ void __launch_bounds__(256) gate_kernel(const T *__restrict__ k, cons
 #pragma unroll
             for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);  // stays in the group
             if (gl == 0 && r < rows) {
-                alpha[r] = gate_alpha(beta[r], s, euler);
+                alpha[r] = gate_alpha(bt[u], s, euler);
                 if (lambda) lambda[r] = s;
             }
         }
