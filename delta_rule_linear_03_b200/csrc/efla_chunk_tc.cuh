@@ -382,6 +382,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Launched as a programmatic dependent of the grid before it (the prep
+    // kernel, or the segment chain): the prologue above overlaps that grid's
+    // last wave; nothing it wrote is read before this wait returns.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp < 8) {
         // ------------------------------------------------------------ TMEM <-> smem warps
@@ -416,54 +420,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&bar[B_SBFULL]);
         }
-        // Only the 256-thread vote on barrier 2 leaves the loop: a failed wait
-        // inside one group (barriers 1 and 3) skips that group's work, and the
-        // abort flag it set makes the next vote leave.
+        // A state-row warp (quads 2, 3) leaves the loop on its own when a wait
+        // fails: no barrier inside the loop ties it to the others.  The O
+        // warps (quads 0, 1) share the staging tile through named barrier 3,
+        // so they leave together, on the vote taken before it.  A failed wait
+        // sets the abort flag, which makes every other wait give up at once.
         for (int n = 0; n < ncj; ++n) {
             const int b = n & 1;
             const uint32_t ty = T_Y + 64 * b + c0;
-            bool bad = false;
             if (dwarp) {
                 // D = U + (-W S): TMEM lanes 64..127 of Y, plus U from the stage
                 const int c = row - 64;
                 // (the stage's own barrier too: U landed by the bulk copy is
                 // visible to the threads that observe that barrier's phase)
-                bool ok = mbar_wait(&bar[B_DFULL], n & 1, abort_flag);
+                if (!mbar_wait(&bar[B_DFULL], n & 1, abort_flag)) break;
                 if (row == 64 && cpart == 0) EFLA_TR(28, n);
-                ok = ok && mbar_wait(&bar[B_FULLB + b], (n >> 1) & 1, abort_flag);
+                if (!mbar_wait(&bar[B_FULLB + b], (n >> 1) & 1, abort_flag)) break;
                 if (row == 64 && cpart == 0) EFLA_TR(10, n);
-                bad = bar_any(1, 128, !ok || *abort_flag);
-                if (!bad) {
-                    tc_fence_after();
-                    uint32_t r[32];
-                    tmem_ld32(tl + ty, r);
-                    const unsigned char *urow = sm + b * STAGE + SL_U * SLOT + c * 256;
-                    float u[32];
+                tc_fence_after();
+                uint32_t r[32];
+                tmem_ld32(tl + ty, r);
+                const unsigned char *urow = sm + b * STAGE + SL_U * SLOT + c * 256;
+                float u[32];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float4 v =
-                            *reinterpret_cast<const float4 *>(urow + (((uint32_t)(8 * cpart + j) ^ (c & 15)) << 4));
-                        u[4 * j] = v.x;
-                        u[4 * j + 1] = v.y;
-                        u[4 * j + 2] = v.z;
-                        u[4 * j + 3] = v.w;
-                    }
-                    tmem_ld_wait(r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] = u[i] + __uint_as_float(r[i]);
-                    write_split32(sm + OFF_DB + b * 2 * SLOT, SLOT, c, 4 * cpart, x);
-                    fence_proxy_async();
-                    tc_fence_before();
-                    mbar_arrive(&bar[B_DELTA]);
-                    if (row == 64 && cpart == 0) EFLA_TR(11, n);
+                for (int j = 0; j < 8; ++j) {
+                    const float4 v =
+                        *reinterpret_cast<const float4 *>(urow + (((uint32_t)(8 * cpart + j) ^ (c & 15)) << 4));
+                    u[4 * j] = v.x;
+                    u[4 * j + 1] = v.y;
+                    u[4 * j + 2] = v.z;
+                    u[4 * j + 3] = v.w;
                 }
+                tmem_ld_wait(r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = u[i] + __uint_as_float(r[i]);
+                write_split32(sm + OFF_DB + b * 2 * SLOT, SLOT, c, 4 * cpart, x);
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(&bar[B_DELTA]);
+                if (row == 64 && cpart == 0) EFLA_TR(11, n);
             }
-            const bool ok = !bad && mbar_wait(&bar[B_SFULL], n & 1, abort_flag);
+            const bool ok = mbar_wait(&bar[B_SFULL], n & 1, abort_flag);
             if (row == 64 && cpart == 0) EFLA_TR(12, n);
-            if (bar_any(2, 256, !ok || *abort_flag)) break;
-            if (row == 64 && cpart == 0) EFLA_TR(29, n);
-            tc_fence_after();
-            {
+            if (!ok && dwarp) break;
+            if (ok) {
+                tc_fence_after();
                 uint32_t r[32];
                 tmem_ld32(tl + T_S + c0, r);
                 tmem_ld_wait(r);
@@ -476,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bar[B_SBFULL]);
                 if (row == 64 && cpart == 0) EFLA_TR(13, n);
             }
-            if (n == ncj - 1 && job.sl) {
+            if (ok && n == ncj - 1 && job.sl) {
                 float *dst = job.sl + ((size_t)bh * DK + row) * DK + j0 + c0;
 #pragma unroll
                 for (int c = 0; c < 32; c += 4)
@@ -487,9 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // store (rows past L are clipped by the tensor map).  The staging
                 // tile is rewritten only after the previous store has read it.
                 const bool storer = warp == 0 && lane == 0;
-                const bool okO = mbar_wait(&bar[B_OFULL + b], (n >> 1) & 1, abort_flag);
+                const bool okO = ok && mbar_wait(&bar[B_OFULL + b], (n >> 1) & 1, abort_flag);
                 if (storer) bulk_wait_read0();
-                if (!bar_any(3, 128, !okO || *abort_flag)) {
+                if (bar_any(3, 128, !okO || *abort_flag)) break;
+                {
                     tc_fence_after();
                     uint32_t r[32];
                     tmem_ld32(tl + ty, r);
@@ -729,6 +731,9 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     const int t0 = chunk * C, n = min(C, L - t0);
     const size_t row0 = (size_t)bh * L + t0;
     if (p == 0) EFLA_TR(49, 1023);
+    // the serial kernel may be scheduled once every prep CTA is running (it
+    // waits for this grid's completion before reading the workspace)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (p == 0) {
         *abort_flag = 0;
         for (int i = 0; i < 6; ++i) mbar_init(&bar[i], 1);
@@ -1127,9 +1132,20 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
     const int P = segments(bh, nc);
     auto run = [&](const SegPlan &plan) {
-        chunk_tc_kernel<Tout><<<dim3((unsigned)grid, (unsigned)plan.njobs), kThreads, SMEM_BYTES, st>>>(mq, mk, mo,
-                                                                                                      img, plan);
-        return cudaGetLastError() == cudaSuccess;
+        // programmatic stream serialisation: the CTAs may start (and run
+        // their prologue) before the previous grid has finished
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid, (unsigned)plan.njobs);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const unsigned char *cimg = img;
+        return cudaLaunchKernelEx(&cfg, chunk_tc_kernel<Tout>, mq, mk, mo, cimg, plan) == cudaSuccess;
     };
     SegPlan plan{};
     plan.nc = nc;
