@@ -305,8 +305,6 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until every committed bulk store of this thread has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Wait until every committed bulk store of this thread has completed.
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // cp.async.bulk shared -> global of `bytes` (multiple of 16, both ends
 // 16-byte aligned), in this thread's bulk async group.
@@ -660,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lastB[s] >= 0) mbar_wait(&bar[B_FULLB + s], (lastB[s] >> 1) & 1, &never);
         }
     }
-    if (threadIdx.x == 0) bulk_wait0();  // the O stores this thread issued are complete
+    if (threadIdx.x == 0) bulk_wait_read0();  // the O stores this thread issued have read the staging tile
     __syncwarp();
     tc_fence_before();
     __syncthreads();
@@ -676,8 +674,10 @@ constexpr int kCopyThread = 224;  // lane 0 of warp 7, idle during the diagonal 
 // Shared memory of one prep CTA (base aligned to 1024 B):
 //   [0, 32K)   K0 Q0 K1 Q1 (64 x 64 bf16 boxes, 128-byte swizzle): [K; Q] is
 //              the 128-row A operand of [K; Q] K^T per d_k half, K also its B;
-//              V0 and V1 later land over Q0 and Q1
-//   [32K, 48K) A (fp32, Sw64), then T in place, then T' hi and lo boxes
+//              V0 and V1 later land over Q0 and Q1; -W is staged over K0 and
+//              K1, then U's second half over V0 and V1
+//   [32K, 48K) A (fp32, Sw64), then T in place, then T' hi and lo boxes,
+//              then U's first half
 //   [48K, 52K) A's diagonal blocks (diag_index), then scratch of the solve
 constexpr uint32_t P_KQ = 0, P_AT = 4 * SLOT, P_AD = 6 * SLOT, P_ALPHA = P_AD + 4096, P_BAR = P_ALPHA + 256;
 constexpr uint32_t P_SMEM = P_BAR + 64 + 1024;  // + barriers, TMEM slot, abort flag; + alignment slack
@@ -758,6 +758,9 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     // bounded wait by every thread; the answer is block-uniform
     auto wait_all = [&](int i, uint32_t parity) { return !__syncthreads_or(!mbar_wait(&bar[i], parity, abort_flag)); };
     bool issued_v = false, issued_mma = false;  // (copy thread / thread 0) for the drain after a failure
+    // beta of the key row this thread gates (four lanes per row, lane 0 of
+    // each four loads it), fetched while K and Q are still landing
+    const float beta_r = ((p & 3) == 0 && (p >> 2) < n) ? beta[row0 + (p >> 2)] : 0.f;
     bool ok = wait_all(0, 0);
     if (p == 0) EFLA_TR(50, 1023);
     if (p == 0 && ok) {  // G = [K; Q] K^T: 8 k-steps over d_k
@@ -786,7 +789,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
         float ss = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
         ss += __shfl_xor_sync(0xffffffffu, ss, 1);
         ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-        if (h == 0) alpha[r] = (r < n) ? gate_alpha(beta[row0 + r], ss, euler != 0) : 0.f;
+        if (h == 0) alpha[r] = (r < n) ? gate_alpha(beta_r, ss, euler != 0) : 0.f;
     }
     ok = ok && wait_all(2, 0);  // (also publishes alpha)
     tc_fence_after();
@@ -800,20 +803,31 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
         tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + 32 * cpart, r32);
         tmem_ld_wait(r32);
         if (quad < 2) {
-            const int i = 32 * quad + lane;
+            // row i (block b = i / 16) against the warp's two 16-column blocks
+            // bj = 2 cpart, 2 cpart + 1: the diagonal block goes to Ad (its
+            // strictly lower part, fp32, one column m at a time: diag_index
+            // steps by 16 per column), blocks left of it to AT (only ever a TF32
+            // operand: stored rounded, four columns at a time), blocks right of
+            // it nowhere
+            const int i = 32 * quad + lane, b = i >> 4, rl = i & 15;
             const float ai = alpha[i];
+            float *adr = Ad + diag_index(b, 0, rl & 1, rl >> 1);
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-                const int j = 32 * cpart + x;
-                const float a0 = (j < i) ? ai * __uint_as_float(r32[x]) : 0.f;
-                const float a1 = (j + 1 < i) ? ai * __uint_as_float(r32[x + 1]) : 0.f;
-                if ((j >> 4) == (i >> 4)) {
-                    const int b = i >> 4, m = j & 15, rl = i & 15;
-                    Ad[diag_index(b, m, rl & 1, rl >> 1)] = a0;
-                    Ad[diag_index(b, m + 1, rl & 1, rl >> 1)] = a1;
-                } else if ((j >> 4) < (i >> 4)) {  // only ever a TF32 operand: stored rounded
-                    *reinterpret_cast<float2 *>(AT.at(i, j)) =
-                        make_float2(__uint_as_float(f2tf32(a0)), __uint_as_float(f2tf32(a1)));
+            for (int xb = 0; xb < 2; ++xb) {
+                const int bj = 2 * cpart + xb;
+                if (bj == b) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) adr[16 * m] = (m < rl) ? ai * __uint_as_float(r32[16 * xb + m]) : 0.f;
+                } else if (bj < b) {
+#pragma unroll
+                    for (int m = 0; m < 16; m += 4) {
+                        const uint32_t *g = &r32[16 * xb + m];
+                        *reinterpret_cast<float4 *>(AT.at(i, 16 * bj + m)) =
+                            make_float4(__uint_as_float(f2tf32(ai * __uint_as_float(g[0]))),
+                                        __uint_as_float(f2tf32(ai * __uint_as_float(g[1]))),
+                                        __uint_as_float(f2tf32(ai * __uint_as_float(g[2]))),
+                                        __uint_as_float(f2tf32(ai * __uint_as_float(g[3]))));
+                    }
                 }
             }
         } else {
@@ -931,7 +945,6 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
         bulk_store(out + IMG_W + SLOT, sm + P_KQ + 2 * SLOT, SLOT);
         bulk_commit();
         issue_wu(SLOT, 4);
-        bulk_wait_read0();  // the K boxes are reused for U below
     }
     ok = ok && wait_all(4, 0);
     tc_fence_after();
@@ -941,8 +954,10 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
             uint32_t r32[32];
             tmem_ld32(tq + 32 * h, r32);
             tmem_ld_wait(r32);
-            if (wlane) {  // staged: half 0 over T', half 1 over the K0 and V0 boxes
-                unsigned char *dst = sm + (cpart ? P_KQ : P_AT) + wrow * 256;
+            if (wlane) {  // staged: half 0 over T', half 1 over V0 (rows 0-31) and V1 (rows 32-63),
+                          // all free once U is done; the K boxes may still be in the W store
+                unsigned char *dst = cpart ? sm + P_KQ + SLOT + (wrow >> 5) * 2 * SLOT + (wrow & 31) * 256
+                                           : sm + P_AT + wrow * 256;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     *reinterpret_cast<uint4 *>(dst + (((8 * h + c) ^ (wrow & 15)) << 4)) =
@@ -954,10 +969,14 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     __syncthreads();
     if (p == 0 && ok) {
         bulk_store(out + IMG_U, sm + P_AT, UHALF);
-        bulk_store(out + IMG_U + UHALF, sm + P_KQ, UHALF);
+        bulk_store(out + IMG_U + UHALF, sm + P_KQ + SLOT, SLOT);
+        bulk_store(out + IMG_U + UHALF + SLOT, sm + P_KQ + 3 * SLOT, SLOT);
         bulk_commit();
     }
-    if (p == 0 || p == kCopyThread) bulk_wait0();  // the image is written before the CTA exits
+    // shared memory stays valid until every bulk store has read it; the writes
+    // themselves are published by the grid's completion (the serial kernel
+    // reads them after griddepcontrol.wait)
+    if (p == 0 || p == kCopyThread) bulk_wait_read0();
     if (p == 0) EFLA_TR(54, 1023);
     if (!ok) {
         // after a failed wait: every TMA load issued lands and every product
