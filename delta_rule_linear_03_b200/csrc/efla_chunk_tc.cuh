@@ -175,84 +175,113 @@ struct Sw64 {
     }
 };
 
-// Diagonal 16 x 16 blocks of A, laid out for the forward substitution: block
-// b, column m, row parity h, then the 8 rows 2s + h (s = 0..7) contiguous.
-__device__ __forceinline__ int diag_index(int b, int m, int h, int s) { return ((b * 16 + m) * 2 + h) * 8 + s; }
+// Diagonal 16 x 16 blocks of A, laid out for the forward substitution:
+// block b, column m, then its 16 rows r contiguous.
+__device__ __forceinline__ int diag_index(int b, int m, int r) { return (b * 16 + m) * 16 + r; }
+
+// One 16 x 8 tile product on mma.sync, acc += X[r0 + 0..15][k0 + 0..7] Y[k0 + 0..7][n0 + 0..7]
+// (TF32 operands, fp32 accumulation; g = lane / 4, t = lane % 4 as in the
+// m16n8k8 fragment layout).  xa(r, k) and yb(k, n) return TF32 bit patterns.
+template <typename XA, typename YB>
+__device__ __forceinline__ void tile_mma(float (&acc)[4], int g, int t, int r0, int k0, int n0, XA xa, YB yb) {
+    const uint32_t a[4] = {xa(r0 + g, k0 + t), xa(r0 + g + 8, k0 + t), xa(r0 + g, k0 + t + 4),
+                           xa(r0 + g + 8, k0 + t + 4)};
+    const uint32_t b[2] = {yb(k0 + t, n0 + g), yb(k0 + t + 4, n0 + g)};
+    mma_tf32(acc, a, b);
+}
 
 // T = (I + A)^{-1} for the strictly lower triangular 64 x 64 A, in place:
-// AT holds A's blocks left of the diagonal (rounded to TF32) on entry and T's lower triangle
-// (diagonal blocks included) on return.  First the four 16 x 16 diagonal
-// blocks by right-looking forward substitution (warps 0-3, one block each,
-// one column per lane pair, fp32, A's diagonal blocks read from their own
-// copy Ad); then block rows I = 1..3:
-//     R = A_{I,<I} T_{<I,<I},   T_{I,<I} = -T_II R,
-// as 16 x 8 tiles on mma.sync (TF32 operands, fp32 accumulation), warp w
-// owning column tile w.  TF32 here costs nothing measurable: T then feeds
-// bf16 hi/lo operands, and an emulation of the whole computation gave the
-// same error against the oracle with fp32 or TF32 block products.  Every R
-// of a block row is formed (and parked in Ad, free by then) before any of
-// its T tiles overwrites the A tiles the others still read.  NT = 256
-// threads call it together; it ends with all of them synchronised.
+// AT holds A's blocks left of the diagonal (rounded to TF32) on entry and T's
+// lower triangle (diagonal blocks included, zeros above them) on return; A's
+// diagonal blocks come in their own copy Ad.
+//   1. The four 16 x 16 diagonal blocks by forward substitution in fp32,
+//      one column per lane (warps 0-1): step m takes T[m][c], final by then
+//      in the lane's own registers, times column m of A.
+//   2. The lower-left 16 x 16 block of each 32 x 32 diagonal block
+//      (2 x 2 block inverse):  T21 = -T22 (A21 T11)      (warps 0-3)
+//   3. The lower-left 32 x 32 block:  T_lower = -T2 (A21 T1), T1 and T2 the
+//      32 x 32 diagonal blocks finished by 1 and 2         (warps 0-7)
+// Products 2 and 3 run as 16 x 8 tiles on mma.sync with TF32 operands and
+// fp32 accumulation, skipping the k-steps where T is zero.  TF32 here costs
+// nothing measurable: T then feeds bf16 hi/lo operands, and an emulation of
+// the whole computation gave the same error against the oracle with fp32
+// or TF32 block products.  Each inner product A21 T is formed (and parked
+// in Ad, free by then) before its result overwrites the A tile it read.
+// NT = 256 threads call it together; it ends with all of them synchronised.
 template <int NT>
 __device__ __forceinline__ void invert_unit_lower(const int p, float *__restrict__ Ad, const Sw64 AT) {
-    static_assert(NT / 32 >= 6, "one warp per column tile of the last block row");
-    if (p < 128) {
-        const int w = p >> 5, l = p & 31, c = l & 15, h = l >> 4, base = 16 * w;
-        float acc[8];
+    static_assert(NT == 256, "eight warps: one per 16 x 8 tile of the last step");
+    const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
+    const auto at_tf32 = [&](int r, int c) { return f2tf32(*AT.at(r, c)); };        // T (fp32)
+    const auto at_raw = [&](int r, int c) { return __float_as_uint(*AT.at(r, c)); };  // A (stored as TF32)
+    // 1. diagonal blocks
+    if (p < 64) {
+        const int blk = p >> 4, c = p & 15, base = 16 * blk;
+        float x[16];
 #pragma unroll
-        for (int s = 0; s < 8; ++s) acc[s] = (2 * s + h == c) ? 1.f : 0.f;
+        for (int r = 0; r < 16; ++r) x[r] = (r == c) ? 1.f : 0.f;
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const float x = __shfl_sync(0xffffffffu, acc[m >> 1], ((m & 1) << 4) | c);
-            const float4 a0 = *reinterpret_cast<const float4 *>(Ad + diag_index(w, m, h, 0));
-            const float4 a1 = *reinterpret_cast<const float4 *>(Ad + diag_index(w, m, h, 4));
-            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        for (int m = 0; m < 15; ++m) {
+            const float4 *col = reinterpret_cast<const float4 *>(Ad + diag_index(blk, m, 0));
+            float a[16];
 #pragma unroll
-            for (int s = 0; s < 8; ++s) acc[s] = fmaf(-a[s], x, acc[s]);
+            for (int q = 0; q < 4; ++q) {
+                const float4 v = col[q];
+                a[4 * q] = v.x, a[4 * q + 1] = v.y, a[4 * q + 2] = v.z, a[4 * q + 3] = v.w;
+            }
+#pragma unroll
+            for (int r = m + 1; r < 16; ++r) x[r] = fmaf(-a[r], x[m], x[r]);
         }
 #pragma unroll
-        for (int s = 0; s < 8; ++s) *AT.at(base + 2 * s + h, base + c) = acc[s];
+        for (int r = 0; r < 16; ++r) *AT.at(base + r, base + c) = x[r];
     }
     ptx::named_bar(1, NT);
     if (p == 0) EFLA_TR(55, 1023);
-    const int w = p >> 5, lane = p & 31, g = lane >> 2, t = lane & 3;
-    float *park = Ad + w * 128;  // this warp's 16 x 8 R tile, row-major
-#pragma unroll 1
-    for (int I = 1; I < 4; ++I) {
-        const int r0 = 16 * I, c0 = 8 * w;
-        const bool mine = w < 2 * I;
-        if (mine) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            // R tile = A[r0.., k] T[k, c0..] over k from the column's own block up to r0
-#pragma unroll 1
-            for (int k0 = 16 * (w >> 1); k0 < r0; k0 += 8) {
-                // A's tiles are stored already rounded to TF32
-                const uint32_t a[4] = {__float_as_uint(*AT.at(r0 + g, k0 + t)), __float_as_uint(*AT.at(r0 + g + 8, k0 + t)),
-                                       __float_as_uint(*AT.at(r0 + g, k0 + t + 4)),
-                                       __float_as_uint(*AT.at(r0 + g + 8, k0 + t + 4))};
-                const uint32_t bb[2] = {f2tf32(*AT.at(k0 + t, c0 + g)), f2tf32(*AT.at(k0 + t + 4, c0 + g))};
-                mma_tf32(acc, a, bb);
-            }
-            *reinterpret_cast<float2 *>(park + g * 8 + 2 * t) = make_float2(acc[0], acc[1]);
-            *reinterpret_cast<float2 *>(park + (g + 8) * 8 + 2 * t) = make_float2(acc[2], acc[3]);
-        }
-        ptx::named_bar(1, NT);  // every R formed: block row I of A may now be overwritten
-        if (mine) {
-            float out[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {  // T tile = -T_II R tile
-                const int k0 = r0 + 8 * kk;
-                const uint32_t a[4] = {f2tf32(*AT.at(r0 + g, k0 + t)), f2tf32(*AT.at(r0 + g + 8, k0 + t)),
-                                       f2tf32(*AT.at(r0 + g, k0 + t + 4)), f2tf32(*AT.at(r0 + g + 8, k0 + t + 4))};
-                const uint32_t bb[2] = {f2tf32(park[(8 * kk + t) * 8 + g]), f2tf32(park[(8 * kk + t + 4) * 8 + g])};
-                mma_tf32(out, a, bb);
-            }
-            *reinterpret_cast<float2 *>(AT.at(r0 + g, c0 + 2 * t)) = make_float2(-out[0], -out[1]);
-            *reinterpret_cast<float2 *>(AT.at(r0 + g + 8, c0 + 2 * t)) = make_float2(-out[2], -out[3]);
-        }
-        ptx::named_bar(1, NT);
-        if (p == 0) EFLA_TR(55 + I, 1023);
+    // 2. T21 of the 32 x 32 block h (rows 32 h + 16 .., columns 32 h ..), column tile nt
+    float *park2 = Ad + (w >> 1) * 256;  // R = A21 T11 of block h, 16 x 16 row-major
+    if (p < 128) {
+        const int base = 32 * (w >> 1), nt = w & 1;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k0 = 8 * nt; k0 < 16; k0 += 8)  // T11[k][8 nt + j] = 0 for k < 8 nt
+            tile_mma(acc, g, t, 16, k0, 8 * nt, [&](int r, int k) { return at_raw(base + r, base + k); },
+                     [&](int k, int n) { return at_tf32(base + k, base + n); });
+        *reinterpret_cast<float2 *>(park2 + g * 16 + 8 * nt + 2 * t) = make_float2(acc[0], acc[1]);
+        *reinterpret_cast<float2 *>(park2 + (g + 8) * 16 + 8 * nt + 2 * t) = make_float2(acc[2], acc[3]);
     }
+    ptx::named_bar(1, NT);
+    if (p < 128) {
+        const int base = 32 * (w >> 1), nt = w & 1;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k0 = 0; k0 < 16; k0 += 8)
+            tile_mma(acc, g, t, 0, k0, 8 * nt, [&](int r, int k) { return at_tf32(base + 16 + r, base + 16 + k); },
+                     [&](int k, int n) { return f2tf32(park2[k * 16 + n]); });
+        *reinterpret_cast<float2 *>(AT.at(base + 16 + g, base + 8 * nt + 2 * t)) = make_float2(-acc[0], -acc[1]);
+        *reinterpret_cast<float2 *>(AT.at(base + 16 + g + 8, base + 8 * nt + 2 * t)) = make_float2(-acc[2], -acc[3]);
+    }
+    ptx::named_bar(1, NT);
+    if (p == 0) EFLA_TR(56, 1023);
+    // 3. rows 32-63, columns 0-31: row tile mt, column tile nt per warp
+    const int mt = w >> 2, nt = w & 3;
+    {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k0 = 8 * nt; k0 < 32; k0 += 8)  // T1[k][8 nt + j] = 0 for k < 8 nt
+            tile_mma(acc, g, t, 32 + 16 * mt, k0, 8 * nt, at_raw, at_tf32);
+        *reinterpret_cast<float2 *>(Ad + (16 * mt + g) * 32 + 8 * nt + 2 * t) = make_float2(acc[0], acc[1]);
+        *reinterpret_cast<float2 *>(Ad + (16 * mt + g + 8) * 32 + 8 * nt + 2 * t) = make_float2(acc[2], acc[3]);
+    }
+    ptx::named_bar(1, NT);
+    if (p == 0) EFLA_TR(57, 1023);
+    {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k0 = 0; k0 < 16 * (mt + 1); k0 += 8)  // T2[16 mt + i][k] = 0 for k >= 16 (mt + 1)
+            tile_mma(acc, g, t, 16 * mt, k0, 8 * nt, [&](int r, int k) { return at_tf32(32 + r, 32 + k); },
+                     [&](int k, int n) { return f2tf32(Ad[k * 32 + n]); });
+        *reinterpret_cast<float2 *>(AT.at(32 + 16 * mt + g, 8 * nt + 2 * t)) = make_float2(-acc[0], -acc[1]);
+        *reinterpret_cast<float2 *>(AT.at(32 + 16 * mt + g + 8, 8 * nt + 2 * t)) = make_float2(-acc[2], -acc[3]);
+    }
+    ptx::named_bar(1, NT);
+    if (p == 0) EFLA_TR(58, 1023);
 }
 
 // bf16 hi + lo split of a pair of fp32 values (hi = rn(x), lo = rn(x - hi)).
@@ -811,7 +840,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
             // it nowhere
             const int i = 32 * quad + lane, b = i >> 4, rl = i & 15;
             const float ai = alpha[i];
-            float *adr = Ad + diag_index(b, 0, rl & 1, rl >> 1);
+            float *adr = Ad + diag_index(b, 0, rl);
 #pragma unroll
             for (int xb = 0; xb < 2; ++xb) {
                 const int bj = 2 * cpart + xb;
