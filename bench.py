@@ -58,11 +58,11 @@ def load_peaks():
 # ------------------------------------------------------------------ algorithmic work
 # DRAM bytes (read + write) of one lm340m efla_chunk_fwd call, summed over its
 # two launches, from one ncu capture of the current kernels
-# (dram__bytes_read.sum + dram__bytes_write.sum; prep 101.25 + 61.9 MB,
-# serial state kernel 184.6 + 40.5 MB).  Well above the 172.5 MB of
-# algorithmic bytes: the prep kernel's per-chunk workspace image (-W, M, U)
-# is written and read back once.
-CHUNK_TRAFFIC_LM340M = 388.3e6
+# (dram__bytes_read.sum + dram__bytes_write.sum, two calls averaged; prep
+# 101.24 + 61.66 MB, serial state kernel 184.60 + 40.95 MB).  Well above the
+# 172.5 MB of algorithmic bytes: the prep kernel's per-chunk workspace image
+# (-W, M, U) is written and read back once.
+CHUNK_TRAFFIC_LM340M = 388.45e6
 
 
 def chunk_bytes(B, H, L, d, esize, esize_o, s0: bool, sl: bool = True):
