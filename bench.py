@@ -50,9 +50,16 @@ def load_peaks():
         j = json.load(open(p))
         return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
                     bf16_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
-                    source="measured")
+                    sm_max_mhz=float(j.get("sm_max_mhz", 1965.0)), source="measured")
     except Exception:
-        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, sm_max_mhz=1965.0, source="fallback")
+
+
+def ffma_peak_tflops(dev, sm_max_mhz):
+    """FP32 FFMA peak derived from unit counts: SMs x 128 fp32 lanes x 2 flop
+    (one fused multiply-add) x the maximum SM clock."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return sms * 128 * 2 * sm_max_mhz * 1e6 / 1e12
 
 
 # ------------------------------------------------------------------ algorithmic work
@@ -344,6 +351,8 @@ def run_ours(args):
         line["backward"] = bench_backward(efla, dev, x, peaks)
     if rank == 0:
         line["gate"] = bench_gate(efla, dev, peaks)
+    if rank == 0 and not args.no_stiffness:
+        line["stiffness_fp32"] = bench_stiffness(efla, dev, peaks)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(efla, dev, x, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -465,6 +474,52 @@ def bench_longctx(efla, dev, peaks, calls=10):
                          "algorithmic_bytes": nbytes, "peak_source": peaks["source"]}}
 
 
+def bench_stiffness(efla, dev, peaks, calls=5):
+    """The stiffness sweep on the exact-fp32 path: B=2, H=16, L=8192, d=128,
+    fp32 q/k/v, ||k|| fixed per run at each of 1e-3, 0.1, 1, 10, 100.  One
+    draw: the keys of each run are the unit keys times ||k||, the same fp32
+    values the workload generator gives for that norm.  Inputs and outputs
+    (0.5 GB) exceed L2; CUDA events over `calls` calls per norm after 2
+    warm-up calls.  The path is bound by fp32 arithmetic, so the roofline is
+    the FFMA peak."""
+    x = workloads.chunk_inputs("stiffness", knorm=1.0)
+    q, k1, v, beta = (x[n].to(dev) for n in ("q", "k", "v", "beta"))
+    B, H, L, d = k1.shape
+    o = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
+    S = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(efla.workspace_size(q.dtype, B, H, L, d, d), dtype=torch.uint8, device=dev)
+    per = {}
+    for kn in workloads.STIFF_KNORMS:
+        k = k1 * kn
+        call = lambda: efla.chunk_fwd(q, k, v, beta, None, o=o, S_L=S, workspace=ws)
+        for _ in range(2):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(calls):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        per[kn] = e0.elapsed_time(e1) / calls
+        del k
+    if efla.last_error() != 0:
+        raise RuntimeError("efla_chunk_fwd reported a device-side error")
+    ms = statistics.mean(per.values())
+    flops = chunk_flops(B, H, L, d)
+    tf = flops / (ms / 1e3) / 1e12
+    peak = ffma_peak_tflops(dev, peaks["sm_max_mhz"])
+    return {"value": B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
+            "ms_per_knorm": {str(kn): t for kn, t in per.items()}, "calls": calls,
+            "config": f"stiffness sweep: B={B} H={H} L={L} d={d} C=64 fp32 q/k/v/o/state, "
+                      f"||k|| in {list(workloads.STIFF_KNORMS)}, beta ~ U(0,1), S0=0",
+            "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "traffic": None, "kernel": "efla_chunk_fwd fp32 path (all launches)",
+                         "algorithmic_flops": flops,
+                         "peak_source": "derived: SMs x 128 fp32 lanes x 2 flop x max SM clock"},
+            "hbm_algorithmic_bytes": chunk_bytes(B, H, L, d, 4, 4, s0=False)}
+
+
 def bench_decode(efla, dev, args, peaks):
     """Decode: batch 64 x 16 heads x d=128 fp32 states, bf16 q/k/v, one
     token per step.  Steps rotate over 4 state sets (256 MB > L2) and are
@@ -555,6 +610,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-longctx", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-stiffness", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
