@@ -218,34 +218,69 @@ __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restri
         sm.S[e] = S0 ? S0[bh * (long)D * D + (long)i * D + j0 + j] : 0.f;
     }
 
-    for (int chunk = 0; chunk < n_chunks; ++chunk) {
-        const int t0 = chunk * C;
-        const int n = min(C, L - t0);
-        const long row0 = bh * (long)L + t0;
+    // The tiles of chunk n+1 (W, K, Q, this CTA's U columns, M) are loaded
+    // into registers while chunk n computes, and moved to shared memory at the
+    // top of the next iteration, so no chunk waits on a global-memory round trip.
+    constexpr int NQ = C * (D / 4) / 256;   // float4s of a C x D tile per thread
+    constexpr int NU = C * (DVT / 4) / 256;  // float4s of the C x DVT U tile per thread
+    constexpr int NM = C * C / 256;          // floats of the C x C M tile per thread
+    static_assert(NQ * 256 == C * (D / 4) && NU * 256 == C * (DVT / 4) && NM * 256 == C * C, "tile split");
+    float4 rw[NQ], rk[NQ], rq[NQ], ru[NU];
+    float rm[NM];
+    auto fetch = [&](int chunk) {
+        const int n = min(C, L - chunk * C);
+        const long row0 = bh * (long)L + chunk * C;
         const long g = bh * n_chunks + chunk;
         const float *Wg = ws.W + g * (size_t)C * D;
         const float *Ug = ws.U + g * (size_t)C * D;
         const float *Mg = ws.M + g * (size_t)C * C;
-        __syncthreads();  // previous chunk's readers are done with the tiles
-        for (int e = t; e < C * (D / 4); e += 256) {
-            const int r = e / (D / 4), c4 = (e % (D / 4)) * 4;
-            float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk;
-            const float4 ww = *reinterpret_cast<const float4 *>(Wg + r * D + c4);
+#pragma unroll
+        for (int x = 0; x < NQ; ++x) {
+            const int e = t + 256 * x, r = e / (D / 4), c4 = (e % (D / 4)) * 4;
+            rw[x] = *reinterpret_cast<const float4 *>(Wg + r * D + c4);
+            rk[x] = rq[x] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (r < n) {
-                kk = load4(k + (row0 + r) * D + c4);
-                qq = load4(q + (row0 + r) * D + c4);
+                rk[x] = load4(k + (row0 + r) * D + c4);
+                rq[x] = load4(q + (row0 + r) * D + c4);
             }
+        }
+#pragma unroll
+        for (int x = 0; x < NU; ++x) {
+            const int e = t + 256 * x, r = e / (DVT / 4), c4 = (e % (DVT / 4)) * 4;
+            ru[x] = *reinterpret_cast<const float4 *>(Ug + r * D + j0 + c4);
+        }
+#pragma unroll
+        for (int x = 0; x < NM; ++x) rm[x] = Mg[t + 256 * x];
+    };
+    auto stash = [&]() {
+#pragma unroll
+        for (int x = 0; x < NQ; ++x) {
+            const int e = t + 256 * x, r = e / (D / 4), c4 = (e % (D / 4)) * 4;
             float *pw = &sm.W[r * LD + c4], *pk = &sm.K[r * LD + c4], *pq = &sm.Q[r * LD + c4];
-            pw[0] = ww.x; pw[1] = ww.y; pw[2] = ww.z; pw[3] = ww.w;
-            pk[0] = kk.x; pk[1] = kk.y; pk[2] = kk.z; pk[3] = kk.w;
-            pq[0] = qq.x; pq[1] = qq.y; pq[2] = qq.z; pq[3] = qq.w;
+            pw[0] = rw[x].x; pw[1] = rw[x].y; pw[2] = rw[x].z; pw[3] = rw[x].w;
+            pk[0] = rk[x].x; pk[1] = rk[x].y; pk[2] = rk[x].z; pk[3] = rk[x].w;
+            pq[0] = rq[x].x; pq[1] = rq[x].y; pq[2] = rq[x].z; pq[3] = rq[x].w;
         }
-        for (int e = t; e < C * DVT / 4; e += 256) {
-            const int r = e / (DVT / 4), c4 = (e % (DVT / 4)) * 4;
-            *reinterpret_cast<float4 *>(&sm.U[r * DVT + c4]) =
-                *reinterpret_cast<const float4 *>(Ug + r * D + j0 + c4);
+#pragma unroll
+        for (int x = 0; x < NU; ++x) {
+            const int e = t + 256 * x, r = e / (DVT / 4), c4 = (e % (DVT / 4)) * 4;
+            *reinterpret_cast<float4 *>(&sm.U[r * DVT + c4]) = ru[x];
         }
-        for (int e = t; e < C * C; e += 256) sm.M[(e / C) * LC + (e % C)] = Mg[e];
+#pragma unroll
+        for (int x = 0; x < NM; ++x) {
+            const int e = t + 256 * x;
+            sm.M[(e / C) * LC + (e % C)] = rm[x];
+        }
+    };
+    if (n_chunks > 0) fetch(0);
+
+    for (int chunk = 0; chunk < n_chunks; ++chunk) {
+        const int t0 = chunk * C;
+        const int n = min(C, L - t0);
+        const long row0 = bh * (long)L + t0;
+        __syncthreads();  // previous chunk's readers are done with the tiles
+        stash();
+        if (chunk + 1 < n_chunks) fetch(chunk + 1);
         __syncthreads();
 
         // D = U - W S and O = Q S: thread owns rows {2 rp, 2 rp + 1}, cols 4 cq..
