@@ -45,14 +45,18 @@ struct PrepSmem {
     static constexpr int LC = kChunk + 1;
     float K[kChunk * LD];
     float V[kChunk * LD];
-    float Q[kChunk * LD];
-    float A[kChunk * LC];   // strictly-lower diag(alpha) K K^T
-    float Tp[kChunk * LC];  // T' = (I + A)^{-1} diag(alpha)
+    union {  // Q is dead once M = Q K^T is formed; A and T' come after it
+        float Q[kChunk * LD];
+        struct {
+            float A[kChunk * LC];   // strictly-lower diag(alpha) K K^T
+            float Tp[kChunk * LC];  // T' = (I + A)^{-1} diag(alpha)
+        };
+    };
     float alpha[kChunk];
 };
 
 template <typename Tin, int D>
-__global__ void __launch_bounds__(256, 1) chunk_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+__global__ void __launch_bounds__(256, 2) chunk_prep_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                                                             const Tin *__restrict__ v,
                                                             const float *__restrict__ beta, int L, int n_chunks,
                                                             SimtScratch ws, bool euler) {
@@ -116,6 +120,7 @@ __global__ void __launch_bounds__(256, 1) chunk_prep_kernel(const Tin *__restric
                 }
         }
         float *Mg = ws.M + g * (size_t)C * C;
+        __syncthreads();  // every thread has read Q: A may now overwrite it
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int r = 4 * tr + u;
