@@ -3,19 +3,27 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one ``efla_chunk_fwd`` over the lm340m workload (B=8, H=8,
-L=2048, d=128, bf16 q/k/v, fp32 beta and state, S0 = 0): gate, UT
-transform, state propagation and intra-chunk output all run inside it.
-The headline ``value`` is chunked-forward tokens/s (B*L per step; a token
-carries all H heads) over all ranks, timed on the device with CUDA events.
-The decode metric (batch 64 x 16 heads x d=128, fp32 states) is reported in
-the ``decode`` object of the same line.
+One step = one ``efla_chunk_fwd`` over the long-context prefill workload
+(B=1, H=16, L=65536, d=128, bf16 q/k/v, fp32 beta, state and o, S0 = 0),
+the largest configuration that the metric is quoted on and that fits one
+GPU: gate, UT transform, state propagation and intra-chunk output all run
+inside it.  The headline ``value`` is chunked-forward tokens/s (B*L per
+step; a token carries all H heads) over all ranks, timed on the device with
+CUDA events around K replays of a CUDA graph of one call.  Its inputs and
+outputs (1.1 GB) are larger than the 126 MB L2, so every step reads them
+from HBM.
 
-Inputs are synthetic and seeded (``workloads``); between timed iterations
-the step rotates over 3 input/output sets (~410 MB, larger than the 126 MB
-L2) so every step reads cold inputs.  Multi-GPU (torchrun, one rank per GPU)
-is weak scaling: every rank runs its own independent (b,h) problems with no
-collective on the data path; time is the max over ranks.
+The same line carries, under ``configs``, every workload of the metric:
+``tiny_d32``, ``lm340m``, ``lm1p3b`` (random S0), ``stiffness`` (all five
+key norms, exact-fp32 path), the long-context prefill (the headline) and
+its 1024-step decode at batch 64 x 16 heads; each with its roofline and a
+CPU baseline (the fp64 oracle at 1 thread and at all host threads, on a
+bounded sample).  ``deltanet_vs_efla`` times the DeltaNet (explicit Euler)
+mode against the exact gate through the same kernels.
+
+Inputs are synthetic and seeded (``workloads``).  Multi-GPU (torchrun, one
+rank per GPU) is weak scaling: every rank runs its own independent (b,h)
+problems with no collective on the data path; time is the max over ranks.
 
 ``--impl reference`` times the fp64 CPU oracle (test infrastructure) on the
 host cores on a bounded sample of the same workload and prints the same
@@ -27,6 +35,7 @@ import argparse
 import json
 import math
 import os
+import platform
 import statistics
 import sys
 import threading
@@ -39,9 +48,9 @@ import torch  # noqa: E402
 
 import workloads  # noqa: E402
 
-WORKLOAD = "lm340m"
+WORKLOAD = "longctx"
 METRIC = "EFLA chunked-fwd tokens/s (% of tensor/HBM roofline); decode tokens/s"
-ROTATE = 3
+PREP_IMAGE_BYTES = 56 * 1024  # per chunk of 64 tokens, tensor-core path workspace image
 
 
 def load_peaks():
@@ -62,19 +71,22 @@ def ffma_peak_tflops(dev, sm_max_mhz):
     return sms * 128 * 2 * sm_max_mhz * 1e6 / 1e12
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
 # ------------------------------------------------------------------ algorithmic work
-# DRAM bytes (read + write) of one lm340m efla_chunk_fwd call, summed over its
-# two launches, from one ncu capture of the current kernels
-# (dram__bytes_read.sum + dram__bytes_write.sum, two calls averaged; prep
-# 101.24 + 61.66 MB, serial state kernel 184.60 + 40.95 MB).  Well above the
-# 172.5 MB of algorithmic bytes: the prep kernel's per-chunk workspace image
-# (-W, M, U) is written and read back once.
-CHUNK_TRAFFIC_LM340M = 388.45e6
-
-
 def chunk_bytes(B, H, L, d, esize, esize_o, s0: bool, sl: bool = True):
-    """Algorithmic HBM bytes of one efla_chunk_fwd: read q, k, v and beta,
-    write o, read S0 (if given) and write S_L once."""
+    """HBM bytes of one efla_chunk_fwd that the method itself needs: read q,
+    k, v and beta, write o, read S0 (if given) and write S_L once.  With o in
+    the q dtype this is the per-unit figure 3 d e + 4 + d e per head-token
+    (1028 B in bf16 at d = 128) plus 64 KB per (b, h) per state read or write."""
     tok = B * H * L
     state = B * H * d * d * 4
     return tok * (3 * d * esize + 4 + d * esize_o) + (state if s0 else 0) + (state if sl else 0)
@@ -90,6 +102,23 @@ def chunk_flops(B, H, L, d, C=64):
 def decode_bytes(B, H, d, esize, esize_o):
     """Read and write the fp32 state once, read q, k, v and beta, write o."""
     return B * H * (2 * 4 * d * d + 3 * d * esize + 4 + d * esize_o)
+
+
+def chunk_launches(efla, dtype, B, H, L, d):
+    """Kernel launches of one efla_chunk_fwd: the tensor-core path runs the
+    prep kernel and one serial launch, or, segment-parallel with P segments,
+    the prep, pass A, P - 2 segment-chain steps and pass B (P + 1 in all).
+    P is read off the workspace size (3 P - 5 fp32 states past the per-chunk
+    images); the CUDA-core path runs two kernels."""
+    ws = efla.workspace_size(dtype, B, H, L, d, d)
+    if dtype != torch.bfloat16 or d != 128:
+        return 2
+    nc = (L + 63) // 64
+    extra = ws - B * H * nc * PREP_IMAGE_BYTES
+    if extra <= 0:
+        return 2
+    P = (extra // (B * H * d * d * 4) + 5) // 3
+    return int(P) + 1
 
 
 # ------------------------------------------------------------------ clocks
@@ -204,34 +233,124 @@ def job_tokens_per_s(world: int, B: int, L: int, steps: int, ms_max: float) -> f
     return world * B * L * steps / (ms_max / 1e3)
 
 
+# ------------------------------------------------------------------ timing helpers
+def graph_of(fn):
+    """Capture one call of ``fn`` into a CUDA graph (after it ran eagerly)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def time_replays(graphs, reps, stream=None):
+    """Mean ms per replay of ``reps`` replays cycling over ``graphs``, CUDA
+    events on the current stream, synchronised on both sides."""
+    stream = stream or torch.cuda.current_stream()
+    for i in range(3):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(reps):
+        graphs[i % len(graphs)].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def hbm_roofline(nbytes, ms, peaks, kernel, traffic=None, note=None):
+    gbs = nbytes / (ms / 1e3) / 1e9
+    r = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s", "frac": gbs / peaks["hbm"],
+         "traffic": traffic, "kernel": kernel, "algorithmic_bytes": nbytes,
+         "peak_source": f"{peaks['source']} (copy bandwidth)"}
+    if note:
+        r["note"] = note
+    return r
+
+
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_rate(x, sample_tokens: int, min_seconds: float, threads: int):
-    """tokens/s of the fp64 oracle on the first ``sample_tokens`` tokens of
-    every (b,h) of ``x`` (a token = one position of one batch row, all heads)."""
+def oracle_rate(x, heads, sample_tokens: int, threads: int, min_seconds: float):
+    """Head-tokens/s of the fp64 oracle on the first ``sample_tokens`` tokens
+    of the (b, h) pairs ``heads`` of ``x``; repeats until ``min_seconds``."""
     import oracle
-    B, H = x["q"].shape[:2]
-    sl = lambda t: t[:, :, :sample_tokens].contiguous()
+    bi = torch.tensor([b for b, _ in heads])
+    hi = torch.tensor([h for _, h in heads])
+    sl = lambda t: t[bi, hi][None, :, :sample_tokens].contiguous()
     q, k, v, beta = (sl(x[n]) for n in ("q", "k", "v", "beta"))
-    oracle.recurrence(q[:1, :1, :8], k[:1, :1, :8], v[:1, :1, :8], beta[:1, :1, :8], threads=1)  # load
+    S0 = None if x.get("S0") is None else x["S0"][bi, hi][None].contiguous()
+    oracle.recurrence(q[:, :1, :4], k[:, :1, :4], v[:, :1, :4], beta[:, :1, :4], threads=1)  # load
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.recurrence(q, k, v, beta, None, threads=threads)
+        oracle.recurrence(q, k, v, beta, S0, threads=threads, want_o=True)
         reps += 1
         dt = time.perf_counter() - t0
-        if dt >= min_seconds or reps >= 50:
+        if dt >= min_seconds or reps >= 1000:
             break
-    return B * sample_tokens * reps / dt, dt, reps
+    return len(heads) * sample_tokens * reps / dt, dt, reps
+
+
+def cpu_baseline_chunk(x, name, seconds=1.5):
+    """The fp64 sequential oracle (C, OpenMP over (b, h)) on a bounded sample
+    of workload ``x``: at all host threads on up to 64 (b, h) pairs, and at
+    one thread on one pair.  tokens/s counts a token as one position of one
+    batch row with all H heads, as the GPU figures do."""
+    import oracle
+    B, H, L, d = x["q"].shape
+    nthreads = oracle.default_threads()
+    pairs = [(b, h) for b in range(B) for h in range(H)][:64]
+    T = max(64, min(L, int(2e9 / (len(pairs) * 6 * d * d * 4))))  # about 0.1-0.5 s per pass
+    rate_n, dt_n, reps_n = oracle_rate(x, pairs, T, nthreads, seconds)
+    T1 = max(64, min(L, int(4e8 / (6 * d * d))))
+    rate_1, dt_1, reps_1 = oracle_rate(x, pairs[:1], T1, 1, seconds)
+    used = min(nthreads, len(pairs))
+    return {"value": rate_n / H, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{name}: first {T} tokens of {len(pairs)} (b,h) pairs x{reps_n} ({dt_n:.1f} s), fp64 "
+                      f"sequential recurrence, OpenMP over (b,h); head-tokens/s / H",
+            "single_thread": {"value": rate_1 / H, "unit": "tokens/s", "cores": 1,
+                              "sample": f"first {T1} tokens of 1 (b,h) pair x{reps_1} ({dt_1:.1f} s)"},
+            "host_threads": nthreads, "cpu_model": cpu_model()}
+
+
+def cpu_baseline_decode(seconds=1.5):
+    """The fp64 oracle's one-token update on the decode batch (64 x 16 states,
+    d = 128) from random states: all host threads on all 1024 states, one
+    thread on 16 of them; tokens/s = batch rows per second."""
+    import oracle
+    Bd, Hd, d = workloads.DECODE_BATCH, workloads.DECODE_HEADS, 128
+    xin = workloads.decode_inputs(1)
+    S = workloads.random_state(Bd, Hd, d).double().numpy()
+    nthreads = oracle.default_threads()
+    out = {}
+    for tag, nb, th in (("all", Bd, nthreads), ("one", 1, 1)):
+        q, k, v, beta = (xin[n][0][:nb] for n in ("q", "k", "v", "beta"))
+        Ss = S[:nb].copy()
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            _, Ss = oracle.decode_step(q, k, v, beta, Ss, threads=th)
+            reps += 1
+            dt = time.perf_counter() - t0
+            if dt >= seconds or reps >= 10000:
+                break
+        out[tag] = (nb * reps / dt, dt, reps)
+    (rn, dtn, repn), (r1, dt1, rep1) = out["all"], out["one"]
+    return {"value": rn, "unit": "tokens/s", "cores": min(nthreads, Bd * Hd), "kind": "oracle",
+            "sample": f"decode: {Bd}x{Hd} states x{repn} steps ({dtn:.1f} s), fp64, OpenMP over (b,h)",
+            "single_thread": {"value": r1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"1x{Hd} states x{rep1} steps ({dt1:.1f} s)"},
+            "host_threads": nthreads, "cpu_model": cpu_model()}
 
 
 def run_reference(args):
-    """The reference arm: the fp64 CPU oracle on the host cores."""
+    """The reference arm: the fp64 CPU oracle on the host cores, on the
+    headline workload; each step is a bounded sample of it (the first 256
+    tokens of every (b, h))."""
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     import oracle
     w = workloads.WORKLOADS[WORKLOAD]
     x = workloads.chunk_inputs(w)
     threads = oracle.default_threads()
-    sample = 64  # one chunk-length of tokens of every (b,h) per step
+    sample = 256
     q, k, v, beta = (x[n][:, :, :sample].contiguous() for n in ("q", "k", "v", "beta"))
     for _ in range(args.warmup):
         oracle.recurrence(q, k, v, beta, None, threads=threads)
@@ -240,15 +359,16 @@ def run_reference(args):
         oracle.recurrence(q, k, v, beta, None, threads=threads)
     dt = time.perf_counter() - t0
     value = w.B * sample * args.steps / dt
+    cores = min(threads, w.B * w.H)
     desc = (f"fp64 sequential oracle, first {sample} tokens of all {w.B}x{w.H} (b,h) of the {WORKLOAD} "
-            f"workload per step, {threads} threads")
+            f"workload per step, {cores} threads ({cpu_model()})")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded, workloads.lm340m distribution)",
+        "data": f"synthetic (seeded, workloads.{WORKLOAD} distribution)",
         "config": workload_config(w, args.gpus),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -256,10 +376,11 @@ def run_reference(args):
 
 
 def workload_config(w, n):
-    return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d={w.d} C=64 {w.dtype} q/k/v, fp32 beta/state/o, S0=0",
+    s0 = "random S0" if w.s0 else "S0=0"
+    return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} d={w.d} C=64 {w.dtype} q/k/v, fp32 beta/state/o, {s0}",
             "B": w.B, "H": w.H, "L": w.L, "head_dim": w.d, "chunk": 64, "global_batch": w.B * n,
             "seq_len": w.L, "parallelism": f"dp{n} (independent (b,h) problems per rank, no collective)",
-            "l2": f"inputs/outputs rotate over {ROTATE} sets (> L2) between timed steps"}
+            "l2": "inputs and outputs (1.1 GB per call) exceed the 126 MB L2"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -272,43 +393,32 @@ def run_ours(args):
     w = workloads.WORKLOADS[WORKLOAD]
     B, H, L, d = w.B, w.H, w.L, w.d
     x = workloads.chunk_inputs(w, seed=rank_seed(w, rank))
-    sets = []
-    for _ in range(ROTATE):
-        s = {n: x[n].to(dev) for n in ("q", "k", "v", "beta")}
-        s["o"] = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
-        s["S"] = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-        sets.append(s)
-    need = efla.workspace_size(x["q"].dtype, B, H, L, d, d)
-    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    launches_per_step = 2 if need else 1
+    q, k, v, beta = (x[n].to(dev) for n in ("q", "k", "v", "beta"))
+    o = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
+    S = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(efla.workspace_size(q.dtype, B, H, L, d, d), 16), dtype=torch.uint8, device=dev)
+    launches_per_step = chunk_launches(efla, q.dtype, B, H, L, d)
     stream = torch.cuda.current_stream(dev)
+    call = lambda: efla.chunk_fwd(q, k, v, beta, None, o=o, S_L=S, workspace=ws)
 
-    def step(i):
-        s = sets[i % ROTATE]
-        efla.chunk_fwd(s["q"], s["k"], s["v"], s["beta"], None, o=s["o"], S_L=s["S"], workspace=ws)
-
-    for i in range(args.warmup):
-        step(i)
+    for _ in range(args.warmup):
+        call()
     torch.cuda.synchronize()
-    # capture one CUDA graph per input set so Python launch overhead stays off the clock
-    graphs = []
-    for r in range(ROTATE):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(r)
-        graphs.append(g)
-    for i in range(max(args.warmup, 3)):
-        graphs[i % ROTATE].replay()
+    g = graph_of(call)  # one call per replay keeps Python launch overhead off the clock
+    for _ in range(args.warmup):
+        g.replay()
     torch.cuda.synchronize()
+    if efla.last_error() != 0:
+        raise RuntimeError("efla_chunk_fwd reported a device-side error")
 
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clk:
+    with ClockSampler(dev.index, period_s=0.001) as clk:
         barrier(world)
         torch.cuda.synchronize()
         clk.active.set()
         e0.record(stream)
-        for i in range(args.steps):
-            graphs[i % ROTATE].replay()
+        for _ in range(args.steps):
+            g.replay()
         e1.record(stream)
         torch.cuda.synchronize()
         clk.active.clear()
@@ -317,51 +427,49 @@ def run_ours(args):
     ms_max = max_over_ranks(ms, world)
     ms_step = ms_max / args.steps
     value = job_tokens_per_s(world, B, L, args.steps, ms_max)
-    del graphs
+    del g
 
-    # roofline of the dominant kernel (the whole efla_chunk_fwd when it is one launch)
-    nbytes = chunk_bytes(B, H, L, d, 2, 4, s0=False)
+    nbytes = chunk_bytes(B, H, L, d, 2, 2, s0=False)  # o counted in the q dtype (bf16)
+    nbytes_f32o = chunk_bytes(B, H, L, d, 2, 4, s0=False)
     flops = chunk_flops(B, H, L, d)
-    achieved_gbs = nbytes / (ms_step / 1e3) / 1e9
     achieved_tf = flops / (ms_step / 1e3) / 1e12
+    roof = hbm_roofline(nbytes, ms_step, peaks, f"efla_chunk_fwd (all {launches_per_step} launches of one call)",
+                        note="bytes count o in the q dtype (bf16), 1028 B per head-token; the call writes o "
+                             "in fp32 (the default output dtype, 1284 B per head-token)")
+    roof["frac_with_fp32_o"] = nbytes_f32o / (ms_step / 1e3) / 1e9 / peaks["hbm"]
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.lm340m distribution)",
+        "vs_baseline": None, "dtype": "bf16", "data": f"synthetic (seeded, workloads.{WORKLOAD} distribution)",
         "config": workload_config(w, world),
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": achieved_gbs / peaks["hbm"],
-                     "traffic": CHUNK_TRAFFIC_LM340M if (WORKLOAD == "lm340m" and launches_per_step == 2) else None,
-                     "kernel": "efla_chunk_fwd (all launches of one call)" if launches_per_step > 1
-                     else "efla_chunk_fwd fused kernel",
-                     "algorithmic_bytes": nbytes, "peak_source": peaks["source"]},
+        "roofline": roof,
         "roofline_tensor": {"achieved": achieved_tf, "peak": peaks["bf16"], "unit": "TFLOP/s",
                             "frac": achieved_tf / peaks["bf16"], "algorithmic_flops": flops,
-                            "peak_source": peaks["source"]},
+                            "peak_source": f"{peaks['source']} (cuBLAS bf16, burst)"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
-
-    if rank == 0 and not args.no_decode:
-        line["decode"] = bench_decode(efla, dev, args, peaks)
-    if rank == 0 and not args.no_longctx:
-        line["longctx_prefill"] = bench_longctx(efla, dev, peaks)
-    if rank == 0 and not args.no_backward:
-        line["backward"] = bench_backward(efla, dev, x, peaks)
-    if rank == 0:
-        line["gate"] = bench_gate(efla, dev, peaks)
-    if rank == 0 and not args.no_stiffness:
-        line["stiffness_fp32"] = bench_stiffness(efla, dev, peaks)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(efla, dev, x, args, world)
+    del q, k, v, beta, o, S, ws
+    torch.cuda.empty_cache()
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        th = oracle.default_threads()
-        rate, dt, reps = oracle_rate(x, sample_tokens=L, min_seconds=10.0, threads=th)
-        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": th, "kind": "oracle",
-                                "sample": f"full {WORKLOAD} workload x{reps} ({dt:.1f} s), fp64 sequential "
-                                          f"recurrence, OpenMP over (b,h)"}
+        line["cpu_baseline"] = cpu_baseline_chunk(x, WORKLOAD)
+    if rank == 0 and world == 1 and not args.no_configs:
+        cfg = {"longctx_prefill": {"value": value / world, "unit": "tokens/s", "ms_per_call": ms_step,
+                                   "config": line["config"]["workload"], "roofline": roof,
+                                   "note": "the headline step", "cpu_baseline": line.get("cpu_baseline")}}
+        for name in ("tiny_d32", "lm340m", "lm1p3b"):
+            cfg[name] = bench_chunk_config(efla, dev, name, peaks, not args.no_cpu_baseline)
+        cfg["stiffness"] = bench_stiffness(efla, dev, peaks, not args.no_cpu_baseline)
+        cfg["longctx_decode"] = bench_decode(efla, dev, peaks, not args.no_cpu_baseline)
+        line["configs"] = cfg
+        line["deltanet_vs_efla"] = bench_modes(efla, dev)
+        line["gate"] = bench_gate(efla, dev, peaks)
+        if not args.no_backward:
+            line["backward"] = bench_backward(efla, dev, peaks)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -371,6 +479,88 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def chunk_case(efla, dev, name, rotate=1, mode="exact", **kw):
+    """Device inputs, outputs and workspace of workload ``name`` (``rotate``
+    independent sets when one set fits in L2) and a list of CUDA graphs of
+    one efla_chunk_fwd call each."""
+    sets, graphs = [], []
+    for r in range(rotate):
+        x = workloads.chunk_inputs(name, seed=None if r == 0 else 500 + r, **kw)
+        B, H, L, d = x["q"].shape
+        t = {n: (x[n].to(dev) if x[n] is not None else None) for n in ("q", "k", "v", "beta", "S0")}
+        t["o"] = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
+        t["S"] = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+        t["ws"] = torch.empty(max(efla.workspace_size(x["q"].dtype, B, H, L, d, d), 16), dtype=torch.uint8,
+                              device=dev)
+        sets.append(t)
+    for t in sets:
+        fn = lambda t=t: efla.chunk_fwd(t["q"], t["k"], t["v"], t["beta"], t["S0"], mode=mode, o=t["o"],
+                                        S_L=t["S"], workspace=t["ws"])
+        fn()
+        torch.cuda.synchronize()
+        graphs.append(graph_of(fn))
+    return sets, graphs
+
+
+def bench_chunk_config(efla, dev, name, peaks, with_cpu, reps=50):
+    """efla_chunk_fwd on one workload at its full size: CUDA graph replays,
+    rotating over independent input sets where one set fits in L2."""
+    w = workloads.WORKLOADS[name]
+    rotate = 3 if name == "lm340m" else 1
+    sets, graphs = chunk_case(efla, dev, name, rotate=rotate)
+    ms = time_replays(graphs, reps)
+    if efla.last_error() != 0:
+        raise RuntimeError("efla_chunk_fwd reported a device-side error")
+    B, H, L, d = w.B, w.H, w.L, w.d
+    es = 2 if w.dtype == "bf16" else 4
+    out = {"value": B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms, "calls": reps,
+           "config": workload_config(w, 1)["workload"],
+           "l2": (f"{rotate} rotating input/output sets (> L2)" if rotate > 1 else
+                  ("inputs and outputs exceed L2" if name != "tiny_d32" else "L2-resident (0.3 MB): latency case")),
+           "gpu_launches_per_call": chunk_launches(efla, w.torch_dtype, B, H, L, d)}
+    if w.dtype == "bf16":
+        out["roofline"] = hbm_roofline(chunk_bytes(B, H, L, d, es, es, s0=w.s0), ms, peaks,
+                                       "efla_chunk_fwd (all launches of one call)",
+                                       note="o counted in the q dtype; the call writes o in fp32")
+        out["roofline"]["frac_with_fp32_o"] = chunk_bytes(B, H, L, d, es, 4, s0=w.s0) / (ms / 1e3) / 1e9 / peaks["hbm"]
+    else:
+        flops = chunk_flops(B, H, L, d)
+        tf = flops / (ms / 1e3) / 1e12
+        peak = ffma_peak_tflops(dev, peaks["sm_max_mhz"])
+        out["roofline"] = {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                           "traffic": None, "kernel": "efla_chunk_fwd exact-fp32 path (all launches)",
+                           "algorithmic_flops": flops,
+                           "peak_source": "derived: SMs x 128 fp32 lanes x 2 flop x max SM clock"}
+    del sets, graphs
+    torch.cuda.empty_cache()
+    if with_cpu:
+        out["cpu_baseline"] = cpu_baseline_chunk(workloads.chunk_inputs(name), name)
+    return out
+
+
+def bench_modes(efla, dev, reps=20):
+    """The pages' one throughput claim is that EFLA trains as fast as
+    DeltaNet.  Both gates run through the same kernels here: the exact gate
+    (EFLA) and alpha = beta (DeltaNet, explicit Euler), timed on lm340m and
+    on the long-context prefill."""
+    out = {}
+    for name in ("lm340m", "longctx"):
+        ms = {}
+        for mode in ("exact", "euler"):
+            sets, graphs = chunk_case(efla, dev, name, rotate=3 if name == "lm340m" else 1, mode=mode)
+            ms[mode] = time_replays(graphs, reps)
+            del sets, graphs
+            torch.cuda.empty_cache()
+        w = workloads.WORKLOADS[name]
+        out[name] = {"efla_ms_per_call": ms["exact"], "deltanet_ms_per_call": ms["euler"],
+                     "efla_tokens_per_s": w.B * w.L / (ms["exact"] / 1e3),
+                     "deltanet_tokens_per_s": w.B * w.L / (ms["euler"] / 1e3),
+                     "efla_over_deltanet_throughput": ms["euler"] / ms["exact"]}
+    if efla.last_error() != 0:
+        raise RuntimeError("efla_chunk_fwd reported a device-side error")
+    return out
 
 
 def bench_gate(efla, dev, peaks, reps=50):
@@ -388,34 +578,20 @@ def bench_gate(efla, dev, peaks, reps=50):
         for (k, b), (a, lam) in zip(sets, outs):
             efla.gate(k, b, alpha=a, lam=lam)
 
-    for _ in range(3):
-        block()
+    block()
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        block()
-    g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / (4 * reps)
+    ms = time_replays([graph_of(block)], reps) / 4
     rows = B * H * L
     nbytes = rows * (2 * d + 4 + 8)  # read k (bf16) and beta, write alpha and lambda
-    gbs = nbytes / (ms / 1e3) / 1e9
     return {"value": rows / (ms / 1e3), "unit": "keys/s", "ms_per_call": ms, "calls": 4 * reps,
             "config": f"lm1p3b keys: {B}x{H}x{L} rows of d={d} bf16, 4 rotating copies (> L2)",
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm"], "traffic": None, "kernel": "gate_kernel",
-                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"]}}
+            "roofline": hbm_roofline(nbytes, ms, peaks, "gate_kernel")}
 
 
-def bench_backward(efla, dev, x, peaks, calls=5):
-    """efla_prefill_bwd on the timed workload (one fp32 dO, no S0/dS_L):
-    exact fp32, one CTA per (b, h) walking the sequence three times."""
+def bench_backward(efla, dev, peaks, calls=5):
+    """efla_prefill_bwd on lm340m (one fp32 dO, no S0/dS_L): exact fp32,
+    one CTA per (b, h) walking the sequence three times."""
+    x = workloads.chunk_inputs("lm340m")
     q, k, v, beta = (x[n].to(dev) for n in ("q", "k", "v", "beta"))
     B, H, L, d = k.shape
     dO = torch.randn(B, H, L, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
@@ -432,56 +608,18 @@ def bench_backward(efla, dev, x, peaks, calls=5):
     if efla.last_error() != 0:
         raise RuntimeError("efla_prefill_bwd reported a device-side error")
     ms = e0.elapsed_time(e1) / calls
-    # HBM bytes: read q, k, v, beta, dO (x2 passes for k); write dq, dk, dv, dbeta; e_t round trip
-    tok = B * H * L
-    nbytes = tok * (3 * d * 2 + 4 + d * 4 + 3 * d * 4 + 4 + 2 * d * 4)
     return {"value": B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms, "calls": calls,
-            "config": f"{WORKLOAD} backward: dq, dk, dv, dbeta, dS0 (fp32), bf16 q/k/v, fp32 dO",
-            "kernel": "backward_kernel (fp32, serial over tokens per (b, h))",
-            "hbm_bytes_estimate": nbytes}
+            "config": "lm340m backward: dq, dk, dv, dbeta, dS0 (fp32), bf16 q/k/v, fp32 dO",
+            "kernel": "backward_kernel (fp32, serial over tokens per (b, h))"}
 
 
-def bench_longctx(efla, dev, peaks, calls=10):
-    """The long-context prefill (B=1, H=16, L=65536, bf16 q/k/v, fp32 o and
-    state): 16 heads leave most SMs idle, so the library runs it
-    segment-parallel.  Same input twice (1.1 GB of inputs and outputs,
-    > L2), CUDA events over `calls` calls after 3 warm-up calls."""
-    x = workloads.chunk_inputs("longctx")
-    q, k, v, beta = (x[n].to(dev) for n in ("q", "k", "v", "beta"))
-    B, H, L, d = k.shape
-    o = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
-    S = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-    ws = torch.empty(efla.workspace_size(q.dtype, B, H, L, d, d), dtype=torch.uint8, device=dev)
-    call = lambda: efla.chunk_fwd(q, k, v, beta, None, o=o, S_L=S, workspace=ws)
-    for _ in range(3):
-        call()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(calls):
-        call()
-    e1.record()
-    torch.cuda.synchronize()
-    if efla.last_error() != 0:
-        raise RuntimeError("efla_chunk_fwd reported a device-side error")
-    ms = e0.elapsed_time(e1) / calls
-    nbytes = chunk_bytes(B, H, L, d, 2, 4, s0=False)
-    gbs = nbytes / (ms / 1e3) / 1e9
-    return {"value": B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms, "calls": calls,
-            "config": f"longctx prefill: B={B} H={H} L={L} d={d} C=64 bf16 q/k/v, fp32 o/state, S0=0",
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm"], "traffic": None, "kernel": "efla_chunk_fwd (all launches)",
-                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"]}}
-
-
-def bench_stiffness(efla, dev, peaks, calls=5):
+def bench_stiffness(efla, dev, peaks, with_cpu, calls=5):
     """The stiffness sweep on the exact-fp32 path: B=2, H=16, L=8192, d=128,
     fp32 q/k/v, ||k|| fixed per run at each of 1e-3, 0.1, 1, 10, 100.  One
     draw: the keys of each run are the unit keys times ||k||, the same fp32
     values the workload generator gives for that norm.  Inputs and outputs
-    (0.5 GB) exceed L2; CUDA events over `calls` calls per norm after 2
-    warm-up calls.  The path is bound by fp32 arithmetic, so the roofline is
-    the FFMA peak."""
+    (0.5 GB) exceed L2; CUDA events over `calls` graph replays per norm.  The
+    path is bound by fp32 arithmetic, so the roofline is the FFMA peak."""
     x = workloads.chunk_inputs("stiffness", knorm=1.0)
     q, k1, v, beta = (x[n].to(dev) for n in ("q", "k", "v", "beta"))
     B, H, L, d = k1.shape
@@ -491,17 +629,9 @@ def bench_stiffness(efla, dev, peaks, calls=5):
     per = {}
     for kn in workloads.STIFF_KNORMS:
         k = k1 * kn
-        call = lambda: efla.chunk_fwd(q, k, v, beta, None, o=o, S_L=S, workspace=ws)
-        for _ in range(2):
-            call()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(calls):
-            call()
-        e1.record()
-        torch.cuda.synchronize()
-        per[kn] = e0.elapsed_time(e1) / calls
+        fn = lambda: efla.chunk_fwd(q, k, v, beta, None, o=o, S_L=S, workspace=ws)
+        fn()
+        per[kn] = time_replays([graph_of(fn)], calls)
         del k
     if efla.last_error() != 0:
         raise RuntimeError("efla_chunk_fwd reported a device-side error")
@@ -509,57 +639,66 @@ def bench_stiffness(efla, dev, peaks, calls=5):
     flops = chunk_flops(B, H, L, d)
     tf = flops / (ms / 1e3) / 1e12
     peak = ffma_peak_tflops(dev, peaks["sm_max_mhz"])
-    return {"value": B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
-            "ms_per_knorm": {str(kn): t for kn, t in per.items()}, "calls": calls,
-            "config": f"stiffness sweep: B={B} H={H} L={L} d={d} C=64 fp32 q/k/v/o/state, "
-                      f"||k|| in {list(workloads.STIFF_KNORMS)}, beta ~ U(0,1), S0=0",
-            "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                         "traffic": None, "kernel": "efla_chunk_fwd fp32 path (all launches)",
-                         "algorithmic_flops": flops,
-                         "peak_source": "derived: SMs x 128 fp32 lanes x 2 flop x max SM clock"},
-            "hbm_algorithmic_bytes": chunk_bytes(B, H, L, d, 4, 4, s0=False)}
+    out = {"value": B * L / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
+           "ms_per_knorm": {str(kn): t for kn, t in per.items()}, "calls": calls,
+           "config": f"stiffness sweep: B={B} H={H} L={L} d={d} C=64 fp32 q/k/v/o/state, "
+                     f"||k|| in {list(workloads.STIFF_KNORMS)}, beta ~ U(0,1), S0=0",
+           "gpu_launches_per_call": 2,
+           "roofline": {"bound": "alu", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                        "traffic": None, "kernel": "efla_chunk_fwd exact-fp32 path (all launches)",
+                        "algorithmic_flops": flops,
+                        "peak_source": "derived: SMs x 128 fp32 lanes x 2 flop x max SM clock"},
+           "hbm_algorithmic_bytes": chunk_bytes(B, H, L, d, 4, 4, s0=False)}
+    del q, k1, v, beta, o, S, ws
+    torch.cuda.empty_cache()
+    if with_cpu:
+        out["cpu_baseline"] = cpu_baseline_chunk(x, "stiffness (||k|| = 1)")
+    return out
 
 
-def bench_decode(efla, dev, args, peaks):
-    """Decode: batch 64 x 16 heads x d=128 fp32 states, bf16 q/k/v, one
-    token per step.  Steps rotate over 4 state sets (256 MB > L2) and are
-    replayed from a CUDA graph of 8 steps."""
+def bench_decode(efla, dev, peaks, with_cpu, reps=3):
+    """The long-context decode: 1024 chained efla_decode_step calls at batch
+    64 x 16 heads x d = 128, fp32 states, bf16 q/k/v, fp32 o, captured as one
+    CUDA graph of the 1024 steps.  The steps rotate over 4 state sets (256 MB,
+    > L2), so every step reads and writes its state in HBM (4 interleaved
+    chains of 256 steps); per-step inputs cycle over 64 drawn sets (0.6% of a
+    step's bytes).  ``single_chain_l2_resident`` times one chain of 1024 steps
+    on one 64 MB state set, which stays in the 126 MB L2 between steps."""
     Bd, Hd, d = workloads.DECODE_BATCH, workloads.DECODE_HEADS, 128
-    nsets = 4
-    xin = workloads.decode_inputs(8)
-    ins = [{n: xin[n][i].to(dev) for n in ("q", "k", "v", "beta")} for i in range(8)]
+    steps, nsets, nin = workloads.DECODE_STEPS, 4, 64
+    xin = workloads.decode_inputs(nin)
+    ins = [{n: xin[n][i].to(dev) for n in ("q", "k", "v", "beta")} for i in range(nin)]
     states = [workloads.random_state(Bd, Hd, d, seed=s).to(dev) for s in range(nsets)]
-    outs = [torch.empty(Bd, Hd, d, dtype=torch.float32, device=dev) for _ in range(8)]
+    outs = [torch.empty(Bd, Hd, d, dtype=torch.float32, device=dev) for _ in range(nin)]
 
-    def block():
-        for i in range(8):
-            efla.decode_step(ins[i]["q"], ins[i]["k"], ins[i]["v"], ins[i]["beta"], states[i % nsets], o=outs[i])
+    def chain(rot):
+        for i in range(steps):
+            a = ins[i % nin]
+            efla.decode_step(a["q"], a["k"], a["v"], a["beta"], states[i % rot], o=outs[i % nin])
 
-    for _ in range(3):
-        block()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        block()
-    reps = max(1, args.steps // 8)
-    for _ in range(3):
-        g.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms_step = e0.elapsed_time(e1) / (8 * reps)
+    res = {}
+    for rot in (nsets, 1):
+        chain(rot)
+        torch.cuda.synchronize()
+        ms = time_replays([graph_of(lambda: chain(rot))], reps) / steps
+        res[rot] = ms
+    if efla.last_error() != 0:
+        raise RuntimeError("efla_decode_step reported a device-side error")
+    ms_step = res[nsets]
     nbytes = decode_bytes(Bd, Hd, d, 2, 4)
-    gbs = nbytes / (ms_step / 1e3) / 1e9
-    return {"value": Bd / (ms_step / 1e3), "unit": "tokens/s", "ms_per_step": ms_step, "steps": 8 * reps,
-            "config": f"batch {Bd} x {Hd} heads x d={d}, fp32 states, bf16 q/k/v, fp32 o, {nsets} state sets (> L2)",
-            "gpu_launches": 8 * reps,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm"], "traffic": None, "kernel": "decode_kernel",
-                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"]}}
+    out = {"value": Bd / (ms_step / 1e3), "unit": "tokens/s", "ms_per_step": ms_step,
+           "steps_per_replay": steps, "replays": reps,
+           "config": f"batch {Bd} x {Hd} heads x d={d}, fp32 states, bf16 q/k/v, fp32 o; one CUDA graph of "
+                     f"{steps} steps over {nsets} rotating state sets (> L2)",
+           "gpu_launches_per_replay": steps,
+           "roofline": hbm_roofline(nbytes, ms_step, peaks, "decode_kernel"),
+           "single_chain_l2_resident": {"value": Bd / (res[1] / 1e3), "unit": "tokens/s", "ms_per_step": res[1],
+                                        "note": "one 64 MB state set: L2-resident between steps"}}
+    del ins, states, outs
+    torch.cuda.empty_cache()
+    if with_cpu:
+        out["cpu_baseline"] = cpu_baseline_decode()
+    return out
 
 
 def bench_e2e(efla, dev, x, args, world):
@@ -584,7 +723,7 @@ def bench_e2e(efla, dev, x, args, world):
     for _ in range(3):
         step()
     torch.cuda.synchronize()
-    n = max(3, min(args.steps, 30))
+    n = max(3, min(args.steps, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     e0.record()
@@ -599,19 +738,51 @@ def bench_e2e(efla, dev, x, args, world):
             "d2h_bytes_per_step": d2h, "steps": n}
 
 
+def run_profile_case(case: str, calls: int):
+    """A few plain calls of one kernel's workload and nothing else, for an
+    ncu capture of that kernel (no timing, no output line)."""
+    import delta_rule_linear_03_b200 as efla
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if case == "gate":
+        x = workloads.chunk_inputs("lm1p3b")
+        k, beta = x["k"].to(dev), x["beta"].to(dev)
+        for _ in range(calls):
+            efla.gate(k, beta)
+    elif case == "decode":
+        Bd, Hd, d = workloads.DECODE_BATCH, workloads.DECODE_HEADS, 128
+        xin = workloads.decode_inputs(calls)
+        states = [workloads.random_state(Bd, Hd, d, seed=s).to(dev) for s in range(4)]
+        for i in range(calls):
+            efla.decode_step(*(xin[n][i].to(dev) for n in ("q", "k", "v", "beta")), states[i % 4])
+    else:
+        x = workloads.chunk_inputs(case)
+        t = {n: (x[n].to(dev) if x[n] is not None else None) for n in ("q", "k", "v", "beta", "S0")}
+        for _ in range(calls):
+            efla.chunk_fwd(t["q"], t["k"], t["v"], t["beta"], t["S0"])
+    torch.cuda.synchronize()
+    if efla.last_error() != 0:
+        raise RuntimeError("device-side error")
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-longctx", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="headline only")
     ap.add_argument("--no-backward", action="store_true")
-    ap.add_argument("--no-stiffness", action="store_true")
+    ap.add_argument("--profile-case", choices=["gate", "decode", "tiny_d32", "lm340m", "lm1p3b", "stiffness",
+                                               "longctx"],
+                    help="run a few plain calls of one workload for an ncu capture, then exit")
+    ap.add_argument("--calls", type=int, default=4, help="calls for --profile-case")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        return run_profile_case(args.profile_case, args.calls)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -136,7 +136,10 @@ def gate(k: torch.Tensor, beta: torch.Tensor, mode: str = "exact", alpha=None, l
         raise ValueError("beta must be float32 [B,H,L]")
     alpha = torch.empty((B, H, L), dtype=torch.float32, device=dev) if alpha is None else alpha
     lam = torch.empty((B, H, L), dtype=torch.float32, device=dev) if lam is None else lam
-    _dev(alpha, lam)
+    for t in (alpha, lam):
+        if t.dtype != torch.float32 or tuple(t.shape) != (B, H, L):
+            raise ValueError("alpha and lambda must be float32 [B,H,L]")
+    _dev(k, alpha, lam)
     with torch.cuda.device(dev):
         _check(_lib.efla_gate(_ptr(k), _dt(k), MODES[mode], _ptr(beta), _ptr(alpha), _ptr(lam),
                               B, H, L, dk, _stream(dev)), "efla_gate")
@@ -148,27 +151,42 @@ def workspace_size(dtype: torch.dtype, B: int, H: int, L: int, d_k: int, d_v: in
     return int(_lib.efla_chunk_fwd_workspace_size(dt, B, H, L, d_k, d_v))
 
 
+def _prefill_args(q, k, v, beta, S0, o, S_L, want_state, out_dtype):
+    """Shape and dtype checks shared by both prefill entry points; returns
+    (device, B, H, L, d_k, d_v, o, S_L) with the outputs allocated when not
+    given.  The C ABI sizes every buffer from B, H, L and d, so a caller
+    buffer of the wrong shape or dtype is refused here, before any launch."""
+    dev = _dev(q, k, v, beta, S0)
+    if k.dim() != 4:
+        raise ValueError("q, k, v must be [B,H,L,d]")
+    B, H, L, dk = k.shape
+    dv = v.shape[-1]
+    if q.shape != k.shape or v.dim() != 4 or v.shape[:3] != (B, H, L) or q.dtype != k.dtype or v.dtype != k.dtype:
+        raise ValueError("q, k, v must share dtype and [B,H,L,*] shape")
+    _dt(q)
+    if beta.dtype != torch.float32 or tuple(beta.shape) != (B, H, L):
+        raise ValueError("beta must be float32 [B,H,L]")
+    if S0 is not None and (S0.dtype != torch.float32 or tuple(S0.shape) != (B, H, dk, dv)):
+        raise ValueError("S0 must be float32 [B,H,d_k,d_v]")
+    if o is None:
+        o = torch.empty((B, H, L, dv), dtype=out_dtype, device=dev)
+    if tuple(o.shape) != (B, H, L, dv) or o.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("o must be float32 or bfloat16 [B,H,L,d_v]")
+    if want_state and S_L is None:
+        S_L = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_L is not None and (S_L.dtype != torch.float32 or tuple(S_L.shape) != (B, H, dk, dv)):
+        raise ValueError("S_L must be float32 [B,H,d_k,d_v]")
+    _dev(q, o, S_L)
+    return dev, B, H, L, dk, dv, o, S_L
+
+
 def chunk_fwd(q, k, v, beta, S0=None, mode: str = "exact", o=None, S_L=None, want_state: bool = True,
               workspace=None, out_dtype=torch.float32):
     """Prefill: q,k [B,H,L,d_k], v [B,H,L,d_v] (one dtype, fp32 or bf16), beta [B,H,L]
     fp32, S0 [B,H,d_k,d_v] fp32 or None.  Returns (o [B,H,L,d_v] in ``out_dtype``
     (or ``o.dtype`` when ``o`` is given), S_L [B,H,d_k,d_v] fp32 or None).
     ``S_L=S0`` updates the state in place."""
-    dev = _dev(q, k, v, beta, S0)
-    B, H, L, dk = k.shape
-    dv = v.shape[-1]
-    if q.shape != k.shape or v.shape[:3] != (B, H, L) or q.dtype != k.dtype or v.dtype != k.dtype:
-        raise ValueError("q, k, v must share dtype and [B,H,L,*] shape")
-    if beta.dtype != torch.float32 or tuple(beta.shape) != (B, H, L):
-        raise ValueError("beta must be float32 [B,H,L]")
-    if S0 is not None and (S0.dtype != torch.float32 or tuple(S0.shape) != (B, H, dk, dv)):
-        raise ValueError("S0 must be float32 [B,H,d_k,d_v]")
-    o = torch.empty((B, H, L, dv), dtype=out_dtype, device=dev) if o is None else o
-    if tuple(o.shape) != (B, H, L, dv):
-        raise ValueError("o must be [B,H,L,d_v]")
-    if want_state and S_L is None:
-        S_L = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
-    _dev(o, S_L)
+    dev, B, H, L, dk, dv, o, S_L = _prefill_args(q, k, v, beta, S0, o, S_L, want_state, out_dtype)
     need = workspace_size(q.dtype, B, H, L, dk, dv)
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -188,17 +206,7 @@ def chunk_fwd_noalloc(q, k, v, beta, S0=None, mode: str = "exact", o=None, S_L=N
     calls on a device; calls that overlap on the GPU race on it).  For hosts
     that cannot let a library allocate.  Outputs are allocated here only when
     not passed in."""
-    dev = _dev(q, k, v, beta, S0)
-    B, H, L, dk = k.shape
-    dv = v.shape[-1]
-    if q.shape != k.shape or v.shape[:3] != (B, H, L) or q.dtype != k.dtype or v.dtype != k.dtype:
-        raise ValueError("q, k, v must share dtype and [B,H,L,*] shape")
-    if beta.dtype != torch.float32 or tuple(beta.shape) != (B, H, L):
-        raise ValueError("beta must be float32 [B,H,L]")
-    o = torch.empty((B, H, L, dv), dtype=out_dtype, device=dev) if o is None else o
-    if want_state and S_L is None:
-        S_L = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
-    _dev(o, S_L)
+    dev, B, H, L, dk, dv, o, S_L = _prefill_args(q, k, v, beta, S0, o, S_L, want_state, out_dtype)
     with torch.cuda.device(dev):
         _check(_lib.efla_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _dt(q), MODES[mode], _ptr(beta),
                                            _ptr(S0), _ptr(o), _dt(o), _ptr(S_L), B, H, L, dk, dv,
@@ -243,8 +251,11 @@ def state_affine(SI, SZ, X, out=None):
         raise ValueError("square states only")
     if out is None:
         out = torch.empty_like(SI)
-    _check(_lib.efla_state_affine(_ptr(SI), _ptr(SZ), _ptr(X), _ptr(out), B, H, d, _stream(dev)),
-           "efla_state_affine")
+    elif out.dtype != torch.float32 or out.shape != SI.shape:
+        raise ValueError("out must be float32 [B,H,d,d]")
+    with torch.cuda.device(dev):
+        _check(_lib.efla_state_affine(_ptr(SI), _ptr(SZ), _ptr(X), _ptr(out), B, H, d, _stream(dev)),
+               "efla_state_affine")
     return out
 
 
@@ -272,10 +283,12 @@ def prefill_bwd(q, k, v, beta, S0, dO, dSL=None, mode: str = "exact", workspace=
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_lib.efla_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _dt(k), MODES[mode], _ptr(beta), _ptr(S0), _ptr(dO),
-                                 _ptr(dSL), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dS0), B, H, L, dk_, dv_,
-                                 _ptr(workspace) if need else None, wbytes if need else 0, _stream(dev)),
-           "efla_prefill_bwd")
+    with torch.cuda.device(dev):
+        _check(_lib.efla_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _dt(k), MODES[mode], _ptr(beta), _ptr(S0),
+                                     _ptr(dO), _ptr(dSL), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbeta), _ptr(dS0),
+                                     B, H, L, dk_, dv_, _ptr(workspace) if need else None,
+                                     wbytes if need else 0, _stream(dev)),
+               "efla_prefill_bwd")
     return dq, dk, dv, dbeta, dS0
 
 

@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/efla.h"
 #include "efla_backward.cuh"
 #include "efla_chunk_simt.cuh"
@@ -19,6 +21,16 @@ using namespace efla;
 namespace {
 
 constexpr long long kMaxElems = (1LL << 46);  // sanity bound on any tensor's element count
+
+// NVTX range around one C-ABI call (validation and launches), so a profiler
+// timeline shows which library call enqueued which kernels.  Header-only
+// NVTX: without an attached tool a push or pop is a test of a null pointer.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -181,6 +193,7 @@ efla_status_t efla_last_error(void) {
 
 efla_status_t efla_gate(const void *k, efla_dtype_t dtype, efla_mode_t mode, const float *beta, float *alpha,
                         float *lambda, int B, int H, int L, int d_k, efla_stream_t stream) {
+    NvtxRange nvtx_("efla_gate");
     efla_status_t s = check_common(dtype, mode);
     if (s != EFLA_OK) return s;
     if (B < 0 || H < 0 || L < 0 || d_k <= 0) return EFLA_ERR_SHAPE;
@@ -222,6 +235,7 @@ efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v, efla_d
                              const float *beta, const float *S0, void *o, efla_dtype_t o_dtype, float *S_L, int B,
                              int H, int L, int d_k, int d_v, void *workspace, size_t workspace_bytes,
                              efla_stream_t stream) {
+    NvtxRange nvtx_("efla_chunk_fwd");
     efla_status_t s = check_common(dtype, mode);
     if (s != EFLA_OK) return s;
     if ((s = check_common(o_dtype, mode)) != EFLA_OK) return s;
@@ -272,6 +286,7 @@ efla_status_t efla_chunk_fwd(const void *q, const void *k, const void *v, efla_d
 efla_status_t efla_decode_step(const void *q, const void *k, const void *v, efla_dtype_t dtype, efla_mode_t mode,
                                const float *beta, float *S, void *o, efla_dtype_t o_dtype, int B, int H, int d_k,
                                int d_v, efla_stream_t stream) {
+    NvtxRange nvtx_("efla_decode_step");
     efla_status_t s = check_common(dtype, mode);
     if (s != EFLA_OK) return s;
     if ((s = check_common(o_dtype, mode)) != EFLA_OK) return s;
@@ -327,6 +342,7 @@ efla_status_t efla_prefill_bwd(const void *q, const void *k, const void *v, efla
                                const float *beta, const float *S0, const float *dO, const float *dSL, float *dq,
                                float *dk, float *dv, float *dbeta, float *dS0, int B, int H, int L, int d_k, int d_v,
                                void *workspace, size_t workspace_bytes, efla_stream_t stream) {
+    NvtxRange nvtx_("efla_prefill_bwd");
     efla_status_t s = check_common(dtype, mode);
     if (s != EFLA_OK) return s;
     if (B < 0 || H < 0 || L < 0) return EFLA_ERR_SHAPE;
@@ -380,6 +396,7 @@ efla_status_t efla_prefill_bwd(const void *q, const void *k, const void *v, efla
 
 efla_status_t efla_state_affine(const float *SI, const float *SZ, const float *X, float *out, int B, int H, int d,
                                 efla_stream_t stream) {
+    NvtxRange nvtx_("efla_state_affine");
     if (B < 0 || H < 0) return EFLA_ERR_SHAPE;
     if (d != 32 && d != 64 && d != 128) return EFLA_ERR_UNSUPPORTED;
     const long long bh = (long long)B * H;
@@ -442,6 +459,7 @@ efla_status_t efla_chunk_fwd_noalloc(const void *q, const void *k, const void *v
                                      efla_mode_t mode, const float *beta, const float *S0, void *o,
                                      efla_dtype_t o_dtype, float *S_L, int B, int H, int L, int d_k, int d_v,
                                      efla_stream_t stream) {
+    NvtxRange nvtx_("efla_chunk_fwd_noalloc");
     efla_status_t s = check_common(dtype, mode);
     if (s != EFLA_OK) return s;
     if ((s = check_common(o_dtype, mode)) != EFLA_OK) return s;

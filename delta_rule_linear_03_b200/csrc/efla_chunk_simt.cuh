@@ -204,10 +204,14 @@ struct StateSmem {
     __align__(16) float S[D * DVT];
 };
 
+// S0 and SL may be the same buffer (in-place state update), so neither is
+// __restrict__.  That case is safe: each CTA reads and writes only its own
+// d_v column slice of its own (b, h), and every read of S0 comes before the
+// first __syncthreads of the chunk loop while SL is written after the last.
 template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
-                                                             const float *__restrict__ S0, Tout *__restrict__ o,
-                                                             float *__restrict__ SL, int L, int n_chunks,
+                                                             const float *S0, Tout *__restrict__ o,
+                                                             float *SL, int L, int n_chunks,
                                                              SimtScratch ws) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     StateSmem<D> &sm = *reinterpret_cast<StateSmem<D> *>(smem_raw);

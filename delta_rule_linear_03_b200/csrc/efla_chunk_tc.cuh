@@ -6,13 +6,16 @@
 // flowchart) chunk by chunk in the UT form of the chunk-parallel scheme that
 // page cites (整体框架, "WY / UT"), with C = 64:
 //
-//   kernel chunk_prep_kernel, one CTA per chunk, all chunks in parallel
+//   kernel chunk_prep_tc_kernel, one CTA per chunk, all chunks in parallel
 //   (everything that does not depend on the state):
 //   alpha = gate(beta, ||k||^2)                       (fp32, CUDA cores)
-//   A  = strictly-lower(diag(alpha) K K^T)            (mma.sync bf16, fp32 acc.)
-//   T  = (I + A)^{-1},  T' = T diag(alpha)            (CUDA cores + mma.sync TF32)
-//   M  = lower-incl-diag(Q K^T)                       (mma.sync bf16)
-//   W  = T' K,  U = T' V                              (mma.sync, T' as bf16 hi + lo)
+//   G  = [K; Q] K^T                                   (tcgen05, M=128 N=64 K=128)
+//   A  = strictly-lower(diag(alpha) K K^T),  M = lower-incl-diag(Q K^T)   (from G)
+//   T  = (I + A)^{-1},  T' = T diag(alpha)            (fp32 substitution on the
+//                                                      diagonal blocks, 2 x 2 block
+//                                                      inverse on TF32 mma.sync)
+//   W  = T' K,  U = T' V                              (tcgen05, M=64 N=128,
+//                                                      T' as bf16 hi + lo)
 //   -> workspace: -W (bf16), M (bf16), U (fp32)
 //   kernel chunk_tc_kernel, serial over the chunks of one (b, h, d_v half):
 //   Y  = [Q; -W] S          ->  [Q S; -W S]           (tcgen05, M=128 N=64 K=128)

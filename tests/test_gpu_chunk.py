@@ -168,3 +168,44 @@ def test_repeatable(efla):
     o1, S1 = run(efla, x)
     o2, S2 = run(efla, x)
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+# ---------------------------------------------------------------- tensor-core path edge cases
+# bf16 q/k/v at d = 128 take the tcgen05 kernels.  Fixed key norms from 1e-3
+# to 100 drive the gate through its small-x limit (alpha -> beta) and its
+# saturation (alpha -> 1/lambda), which changes the scale of A = diag(alpha) K K^T
+# and stresses the TF32 block inverse and the bf16 hi/lo operand splits.
+
+def _tc_segmented(efla, B, H, L):
+    """True when efla_chunk_fwd runs these sizes segment-parallel: the
+    workspace then holds fp32 segment states beyond the per-chunk images
+    (56 KB per chunk of 64 tokens)."""
+    nc = (L + 63) // 64
+    return efla.workspace_size(torch.bfloat16, B, H, L, 128, 128) > B * H * nc * 56 * 1024
+
+
+@pytest.mark.parametrize("knorm", workloads.STIFF_KNORMS)
+@pytest.mark.parametrize("shape", [(2, 4, 700), (1, 2, 3100)], ids=["single_pass", "segmented"])
+def test_stiffness_bf16_tensor_core(efla, knorm, shape):
+    B, H, L = shape
+    assert _tc_segmented(efla, B, H, L) == (L == 3100)
+    x = workloads.chunk_inputs("stiffness", B=B, H=H, L=L, knorm=knorm, dtype="bf16")
+    o, SL = run(efla, x)
+    ro, rS = ref(x)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(SL, rS, "bf16", "S_L")
+
+
+def test_tc_in_place_state_single_pass(efla):
+    """S_L = S0 on the single-pass tensor-core path."""
+    x = workloads.chunk_inputs("lm1p3b", B=2, H=3, L=333)
+    assert not _tc_segmented(efla, 2, 3, 333)
+    S0 = x["S0"]
+    Sg = S0.cuda()
+    o, SL = efla.chunk_fwd(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), x["beta"].cuda(), Sg, S_L=Sg)
+    torch.cuda.synchronize()
+    assert efla.last_error() == 0
+    assert SL.data_ptr() == Sg.data_ptr()
+    ro, rS = ref(x, S0=S0)
+    assert_close(o, ro, "bf16", "o")
+    assert_close(Sg, rS, "bf16", "S_L")

@@ -17,7 +17,8 @@ Workloads (shapes and value distributions):
   {1e-3, 0.1, 1, 10, 100} with a uniformly random direction; beta ~ U(0,1);
   q, v as lm340m (fp32).  S0=0.
 * ``longctx``    B=1 H=16 L=65536 d=128, bf16 prefill as lm340m; then decode
-  steps at batch 64 x 16 heads with fresh q/k/v/beta per step drawn as lm340m.
+  steps at batch 64 x 16 heads with fresh q/k/v/beta per step drawn as lm340m
+  (step s from its own generator, see ``decode_inputs``).
 
 Seeds: ``numpy.random.default_rng(42 + index)`` with index the workload's
 position in ``WORKLOADS``; draw order q, k, v, key-norm scales, beta, S0.
@@ -109,11 +110,15 @@ def _draw_qkv(rng, kind, B, H, L, d, knorm):
 
 
 def chunk_inputs(w: Workload | str, *, B=None, H=None, L=None, knorm=None, seed=None,
-                 s0=None):
+                 s0=None, dtype=None):
     """Inputs of ``efla_chunk_fwd`` for workload ``w`` as CPU torch tensors:
-    dict(q, k, v [B,H,L,d] storage dtype; beta [B,H,L] fp32; S0 [B,H,d,d] fp32 or None)."""
+    dict(q, k, v [B,H,L,d] storage dtype; beta [B,H,L] fp32; S0 [B,H,d,d] fp32 or None).
+    ``dtype`` ("f32" or "bf16") overrides the workload's storage dtype; the
+    values are drawn the same way and then rounded to it."""
     if isinstance(w, str):
         w = WORKLOADS[w]
+    if dtype is not None:
+        w = w.with_(dtype=dtype)
     B = w.B if B is None else B
     H = w.H if H is None else H
     L = w.L if L is None else L
@@ -130,12 +135,24 @@ def chunk_inputs(w: Workload | str, *, B=None, H=None, L=None, knorm=None, seed=
 
 
 def decode_inputs(steps: int, *, B=DECODE_BATCH, H=DECODE_HEADS, d=128, dtype="bf16",
-                  seed=None):
-    """Per-step decode inputs drawn as lm340m: q,k,v [steps,B,H,d], beta [steps,B,H]."""
-    rng = np.random.default_rng(42 + WORKLOADS["longctx"].index + 1000 if seed is None else seed)
-    q, k, v, beta = _draw_qkv(rng, "lm", steps, B, H, d, None)
+                  first: int = 0, seed=None):
+    """Per-step decode inputs drawn as lm340m: q,k,v [steps,B,H,d], beta
+    [steps,B,H], for the steps first .. first+steps-1 of the decode stream.
+    Step s is drawn from its own generator, ``default_rng([base, s])`` with
+    base = 42 + longctx index + 1000, so any window of a long chain (the
+    1024-step long-context decode) is generated without the steps before it."""
+    base = 42 + WORKLOADS["longctx"].index + 1000 if seed is None else seed
+    qs, ks, vs, bs = [], [], [], []
+    for s in range(first, first + steps):
+        rng = np.random.default_rng([base, s])
+        q, k, v, beta = _draw_qkv(rng, "lm", 1, B, H, d, None)  # [1,B,H,d]: one "token" per state
+        qs.append(q.reshape(B, H, d))
+        ks.append(k.reshape(B, H, d))
+        vs.append(v.reshape(B, H, d))
+        bs.append(beta.reshape(B, H))
     dt = torch.float32 if dtype == "f32" else torch.bfloat16
-    return dict(q=_to(q, dt), k=_to(k, dt), v=_to(v, dt), beta=torch.from_numpy(beta))
+    return dict(q=_to(np.stack(qs), dt), k=_to(np.stack(ks), dt), v=_to(np.stack(vs), dt),
+                beta=torch.from_numpy(np.stack(bs)))
 
 
 def random_state(B, H, d, std=0.1, seed=7):
