@@ -50,7 +50,6 @@ import workloads  # noqa: E402
 
 WORKLOAD = "longctx"
 METRIC = "EFLA chunked-fwd tokens/s (% of tensor/HBM roofline); decode tokens/s"
-PREP_IMAGE_BYTES = 56 * 1024  # per chunk of 64 tokens, tensor-core path workspace image
 
 
 def load_peaks():
@@ -114,7 +113,8 @@ def chunk_launches(efla, dtype, B, H, L, d):
     if dtype != torch.bfloat16 or d != 128:
         return 2
     nc = (L + 63) // 64
-    extra = ws - B * H * nc * PREP_IMAGE_BYTES
+    image = efla.workspace_size(dtype, 1, 1, 64, d, d)  # one chunk's image (never segmented)
+    extra = ws - B * H * nc * image
     if extra <= 0:
         return 2
     P = (extra // (B * H * d * d * 4) + 5) // 3

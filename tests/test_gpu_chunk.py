@@ -179,9 +179,10 @@ def test_repeatable(efla):
 def _tc_segmented(efla, B, H, L):
     """True when efla_chunk_fwd runs these sizes segment-parallel: the
     workspace then holds fp32 segment states beyond the per-chunk images
-    (56 KB per chunk of 64 tokens)."""
+    (the workspace of a single chunk is one image)."""
     nc = (L + 63) // 64
-    return efla.workspace_size(torch.bfloat16, B, H, L, 128, 128) > B * H * nc * 56 * 1024
+    image = efla.workspace_size(torch.bfloat16, 1, 1, 64, 128, 128)
+    return efla.workspace_size(torch.bfloat16, B, H, L, 128, 128) > B * H * nc * image
 
 
 @pytest.mark.parametrize("knorm", workloads.STIFF_KNORMS)
