@@ -738,9 +738,11 @@ def bench_e2e(efla, dev, x, args, world):
             "d2h_bytes_per_step": d2h, "steps": n}
 
 
-def run_profile_case(case: str, calls: int):
+def run_profile_case(case: str, calls: int, seq_len=None):
     """A few plain calls of one kernel's workload and nothing else, for an
-    ncu capture of that kernel (no timing, no output line)."""
+    ncu capture of that kernel (no timing, no output line).  ``seq_len``
+    shortens a prefill workload (same heads, same kernels) for captures
+    that would be too large at full length."""
     import delta_rule_linear_03_b200 as efla
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -756,7 +758,7 @@ def run_profile_case(case: str, calls: int):
         for i in range(calls):
             efla.decode_step(*(xin[n][i].to(dev) for n in ("q", "k", "v", "beta")), states[i % 4])
     else:
-        x = workloads.chunk_inputs(case)
+        x = workloads.chunk_inputs(case, L=seq_len)
         t = {n: (x[n].to(dev) if x[n] is not None else None) for n in ("q", "k", "v", "beta", "S0")}
         for _ in range(calls):
             efla.chunk_fwd(t["q"], t["k"], t["v"], t["beta"], t["S0"])
@@ -780,9 +782,10 @@ def main(argv=None):
                                                "longctx"],
                     help="run a few plain calls of one workload for an ncu capture, then exit")
     ap.add_argument("--calls", type=int, default=4, help="calls for --profile-case")
+    ap.add_argument("--profile-len", type=int, default=None, help="sequence length for --profile-case")
     args = ap.parse_args(argv)
     if args.profile_case:
-        return run_profile_case(args.profile_case, args.calls)
+        return run_profile_case(args.profile_case, args.calls, args.profile_len)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -41,15 +41,18 @@ struct SimtScratch {
 
 template <int D>
 struct PrepSmem {
-    static constexpr int LD = D + 1;   // padded row stride of the C x D tiles
-    static constexpr int LC = kChunk + 1;
-    float K[kChunk * LD];
-    float V[kChunk * LD];
+    // Row strides of 16-byte multiples (one 16-byte load reads four
+    // consecutive elements of a row) that are not multiples of 32 words
+    // (rows read together fall in different banks).
+    static constexpr int LD = D + 4;
+    static constexpr int LC = kChunk + 4;
+    __align__(16) float K[kChunk * LD];
+    __align__(16) float V[kChunk * LD];
     union {  // Q is dead once M = Q K^T is formed; A and T' come after it
-        float Q[kChunk * LD];
+        __align__(16) float Q[kChunk * LD];
         struct {
-            float A[kChunk * LC];   // strictly-lower diag(alpha) K K^T
-            float Tp[kChunk * LC];  // T' = (I + A)^{-1} diag(alpha)
+            __align__(16) float A[kChunk * LC];   // strictly-lower diag(alpha) K K^T
+            __align__(16) float Tp[kChunk * LC];  // T' = (I + A)^{-1} diag(alpha)
         };
     };
     float alpha[kChunk];
@@ -81,10 +84,9 @@ __global__ void __launch_bounds__(256, 2) chunk_prep_kernel(const Tin *__restric
             vv = load4(v + (row0 + r) * D + c4);
             qq = load4(q + (row0 + r) * D + c4);
         }
-        float *pk = &sm.K[r * LD + c4], *pv = &sm.V[r * LD + c4], *pq = &sm.Q[r * LD + c4];
-        pk[0] = kk.x; pk[1] = kk.y; pk[2] = kk.z; pk[3] = kk.w;
-        pv[0] = vv.x; pv[1] = vv.y; pv[2] = vv.z; pv[3] = vv.w;
-        pq[0] = qq.x; pq[1] = qq.y; pq[2] = qq.z; pq[3] = qq.w;
+        *reinterpret_cast<float4 *>(&sm.K[r * LD + c4]) = kk;
+        *reinterpret_cast<float4 *>(&sm.V[r * LD + c4]) = vv;
+        *reinterpret_cast<float4 *>(&sm.Q[r * LD + c4]) = qq;
     }
     __syncthreads();
 
@@ -99,24 +101,27 @@ __global__ void __launch_bounds__(256, 2) chunk_prep_kernel(const Tin *__restric
     }
     __syncthreads();
 
-    // 3. A = strictly-lower(diag(alpha) K K^T); M = lower-incl-diag(Q K^T) -> scratch
+    // 3. A = strictly-lower(diag(alpha) K K^T); M = lower-incl-diag(Q K^T) -> scratch.
+    //    Thread: rows 4 tr + u, columns tc + 16 w (u, w < 4); four d_k indices
+    //    per step, each row segment read by one 16-byte load.
     {
-        const int tr = t >> 4, tc = t & 15;  // 4x4 register tile at rows 4tr.., cols 4tc..
+        const int tr = t >> 4, tc = t & 15;
         float g4[4][4] = {}, m4[4][4] = {};
-        for (int i = 0; i < D; ++i) {
-            float a[4], b[4], qa[4];
+#pragma unroll 2
+        for (int i = 0; i < D; i += 4) {
+            float4 a[4], qa[4], b[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                a[u] = sm.K[(4 * tr + u) * LD + i];
-                qa[u] = sm.Q[(4 * tr + u) * LD + i];
-                b[u] = sm.K[(4 * tc + u) * LD + i];
+                a[u] = *reinterpret_cast<const float4 *>(&sm.K[(4 * tr + u) * LD + i]);
+                qa[u] = *reinterpret_cast<const float4 *>(&sm.Q[(4 * tr + u) * LD + i]);
+                b[u] = *reinterpret_cast<const float4 *>(&sm.K[(tc + 16 * u) * LD + i]);
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u)
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    g4[u][w] = fmaf(a[u], b[w], g4[u][w]);
-                    m4[u][w] = fmaf(qa[u], b[w], m4[u][w]);
+                    g4[u][w] = fmaf(a[u].x, b[w].x, fmaf(a[u].y, b[w].y, fmaf(a[u].z, b[w].z, fmaf(a[u].w, b[w].w, g4[u][w]))));
+                    m4[u][w] = fmaf(qa[u].x, b[w].x, fmaf(qa[u].y, b[w].y, fmaf(qa[u].z, b[w].z, fmaf(qa[u].w, b[w].w, m4[u][w]))));
                 }
         }
         float *Mg = ws.M + g * (size_t)C * C;
@@ -124,15 +129,12 @@ __global__ void __launch_bounds__(256, 2) chunk_prep_kernel(const Tin *__restric
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int r = 4 * tr + u;
-            float4 mrow;
-            float *mr = reinterpret_cast<float *>(&mrow);
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-                const int c = 4 * tc + w;
+                const int c = tc + 16 * w;
                 sm.A[r * LC + c] = (c < r) ? sm.alpha[r] * g4[u][w] : 0.f;
-                mr[w] = (c <= r) ? m4[u][w] : 0.f;
+                Mg[r * C + c] = (c <= r) ? m4[u][w] : 0.f;
             }
-            *reinterpret_cast<float4 *>(Mg + r * C + 4 * tc) = mrow;
         }
     }
     __syncthreads();
@@ -158,24 +160,45 @@ __global__ void __launch_bounds__(256, 2) chunk_prep_kernel(const Tin *__restric
     }
     __syncthreads();
 
-    // 5. W = T' K, U = T' V -> scratch.  Thread tile: 4 rows x (D/16) cols.
+    // 5. W = T' K, U = T' V -> scratch.  Thread: rows 4 tr .., columns in
+    //    groups of CW contiguous (CW = 4, or 2 at d = 32): group g starts at
+    //    16 CW g + CW tc, so the 16 threads of a row read one contiguous
+    //    segment.  Four chunk rows m per step (T' row segments by 16-byte
+    //    loads); T' is lower triangular: m < 4 tr + 4.
     {
-        constexpr int CW = D / 16;
+        constexpr int CW = D >= 64 ? 4 : 2, NG = D / (16 * CW), NCW = CW * NG;
         const int tr = t >> 4, tc = t & 15;
-        float w4[4][CW] = {}, u4[4][CW] = {};
-        const int mmax = 4 * tr + 4;  // T' is lower triangular
-        for (int m = 0; m < mmax; ++m) {
-            float a[4];
+        float w4[4][NCW] = {}, u4[4][NCW] = {};
+        auto col = [&](int c) { return 16 * CW * (c / CW) + CW * tc + (c % CW); };
+        const int mmax = 4 * tr + 4;
+        for (int m = 0; m < mmax; m += 4) {
+            float4 a[4];
 #pragma unroll
-            for (int uu = 0; uu < 4; ++uu) a[uu] = sm.Tp[(4 * tr + uu) * LC + m];
+            for (int uu = 0; uu < 4; ++uu) a[uu] = *reinterpret_cast<const float4 *>(&sm.Tp[(4 * tr + uu) * LC + m]);
 #pragma unroll
-            for (int cc = 0; cc < CW; ++cc) {
-                const float kk = sm.K[m * LD + tc + 16 * cc];
-                const float vv = sm.V[m * LD + tc + 16 * cc];
+            for (int v4 = 0; v4 < 4; ++v4) {
+                float kk[NCW], vv[NCW];
+#pragma unroll
+                for (int gg = 0; gg < NG; ++gg) {
+                    const float *kr = &sm.K[(m + v4) * LD + col(CW * gg)];
+                    const float *vr = &sm.V[(m + v4) * LD + col(CW * gg)];
+                    if constexpr (CW == 4) {
+                        const float4 k4 = *reinterpret_cast<const float4 *>(kr), v4v = *reinterpret_cast<const float4 *>(vr);
+                        kk[4 * gg] = k4.x, kk[4 * gg + 1] = k4.y, kk[4 * gg + 2] = k4.z, kk[4 * gg + 3] = k4.w;
+                        vv[4 * gg] = v4v.x, vv[4 * gg + 1] = v4v.y, vv[4 * gg + 2] = v4v.z, vv[4 * gg + 3] = v4v.w;
+                    } else {
+                        const float2 k2 = *reinterpret_cast<const float2 *>(kr), v2 = *reinterpret_cast<const float2 *>(vr);
+                        kk[2 * gg] = k2.x, kk[2 * gg + 1] = k2.y, vv[2 * gg] = v2.x, vv[2 * gg + 1] = v2.y;
+                    }
+                }
 #pragma unroll
                 for (int uu = 0; uu < 4; ++uu) {
-                    w4[uu][cc] = fmaf(a[uu], kk, w4[uu][cc]);
-                    u4[uu][cc] = fmaf(a[uu], vv, u4[uu][cc]);
+                    const float av = v4 == 0 ? a[uu].x : v4 == 1 ? a[uu].y : v4 == 2 ? a[uu].z : a[uu].w;
+#pragma unroll
+                    for (int c = 0; c < NCW; ++c) {
+                        w4[uu][c] = fmaf(av, kk[c], w4[uu][c]);
+                        u4[uu][c] = fmaf(av, vv[c], u4[uu][c]);
+                    }
                 }
             }
         }
@@ -183,9 +206,9 @@ __global__ void __launch_bounds__(256, 2) chunk_prep_kernel(const Tin *__restric
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu)
 #pragma unroll
-            for (int cc = 0; cc < CW; ++cc) {
-                Wg[(4 * tr + uu) * D + tc + 16 * cc] = w4[uu][cc];
-                Ug[(4 * tr + uu) * D + tc + 16 * cc] = u4[uu][cc];
+            for (int c = 0; c < NCW; ++c) {
+                Wg[(4 * tr + uu) * D + col(c)] = w4[uu][c];
+                Ug[(4 * tr + uu) * D + col(c)] = u4[uu][c];
             }
     }
 }
@@ -193,21 +216,37 @@ __global__ void __launch_bounds__(256, 2) chunk_prep_kernel(const Tin *__restric
 template <int D>
 struct StateSmem {
     static constexpr int DVT = 32;       // d_v columns per CTA
-    static constexpr int LD = D + 1;
-    static constexpr int LC = kChunk + 1;
-    float W[kChunk * LD];
-    float K[kChunk * LD];
-    float Q[kChunk * LD];
-    float M[kChunk * LC];
+    // Row strides of 16-byte multiples, so a thread reads four consecutive
+    // elements of a row with one 16-byte load, and not a multiple of 32
+    // words, so the rows a warp reads at once fall in different banks.
+    static constexpr int LD = D + 4;
+    static constexpr int LC = kChunk + 4;
+    __align__(16) float W[kChunk * LD];
+    __align__(16) float K[kChunk * LD];
+    __align__(16) float Q[kChunk * LD];
+    __align__(16) float M[kChunk * LC];
     __align__(16) float U[kChunk * DVT];
     __align__(16) float Dl[kChunk * DVT];
     __align__(16) float S[D * DVT];
 };
 
+__device__ __forceinline__ void fma4(float (&acc)[4], float a, const float4 &b) {
+    acc[0] = fmaf(a, b.x, acc[0]);
+    acc[1] = fmaf(a, b.y, acc[1]);
+    acc[2] = fmaf(a, b.z, acc[2]);
+    acc[3] = fmaf(a, b.w, acc[3]);
+}
+
 // S0 and SL may be the same buffer (in-place state update), so neither is
 // __restrict__.  That case is safe: each CTA reads and writes only its own
 // d_v column slice of its own (b, h), and every read of S0 comes before the
 // first __syncthreads of the chunk loop while SL is written after the last.
+//
+// Per chunk, with every contraction vectorised four elements at a time (one
+// 16-byte load of a row segment feeds 16 FMAs):
+//   D = U - W S,  O = Q S   thread: rows 2 rp, 2 rp + 1; columns 4 cq ..
+//   O += M D                (M lower triangular: m up to the thread's rows)
+//   S += K^T D              thread: d_k rows 4 iq ..; columns 4 jq ..
 template <typename Tin, typename Tout, int D>
 __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                                                              const float *S0, Tout *__restrict__ o,
@@ -232,10 +271,9 @@ __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restri
     // top of the next iteration, so no chunk waits on a global-memory round trip.
     constexpr int NQ = C * (D / 4) / 256;   // float4s of a C x D tile per thread
     constexpr int NU = C * (DVT / 4) / 256;  // float4s of the C x DVT U tile per thread
-    constexpr int NM = C * C / 256;          // floats of the C x C M tile per thread
-    static_assert(NQ * 256 == C * (D / 4) && NU * 256 == C * (DVT / 4) && NM * 256 == C * C, "tile split");
-    float4 rw[NQ], rk[NQ], rq[NQ], ru[NU];
-    float rm[NM];
+    constexpr int NM = C * (C / 4) / 256;    // float4s of the C x C M tile per thread
+    static_assert(NQ * 256 == C * (D / 4) && NU * 256 == C * (DVT / 4) && NM * 256 == C * (C / 4), "tile split");
+    float4 rw[NQ], rk[NQ], rq[NQ], ru[NU], rm[NM];
     auto fetch = [&](int chunk) {
         const int n = min(C, L - chunk * C);
         const long row0 = bh * (long)L + chunk * C;
@@ -259,16 +297,18 @@ __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restri
             ru[x] = *reinterpret_cast<const float4 *>(Ug + r * D + j0 + c4);
         }
 #pragma unroll
-        for (int x = 0; x < NM; ++x) rm[x] = Mg[t + 256 * x];
+        for (int x = 0; x < NM; ++x) {
+            const int e = t + 256 * x, r = e / (C / 4), c4 = (e % (C / 4)) * 4;
+            rm[x] = *reinterpret_cast<const float4 *>(Mg + r * C + c4);
+        }
     };
     auto stash = [&]() {
 #pragma unroll
         for (int x = 0; x < NQ; ++x) {
             const int e = t + 256 * x, r = e / (D / 4), c4 = (e % (D / 4)) * 4;
-            float *pw = &sm.W[r * LD + c4], *pk = &sm.K[r * LD + c4], *pq = &sm.Q[r * LD + c4];
-            pw[0] = rw[x].x; pw[1] = rw[x].y; pw[2] = rw[x].z; pw[3] = rw[x].w;
-            pk[0] = rk[x].x; pk[1] = rk[x].y; pk[2] = rk[x].z; pk[3] = rk[x].w;
-            pq[0] = rq[x].x; pq[1] = rq[x].y; pq[2] = rq[x].z; pq[3] = rq[x].w;
+            *reinterpret_cast<float4 *>(&sm.W[r * LD + c4]) = rw[x];
+            *reinterpret_cast<float4 *>(&sm.K[r * LD + c4]) = rk[x];
+            *reinterpret_cast<float4 *>(&sm.Q[r * LD + c4]) = rq[x];
         }
 #pragma unroll
         for (int x = 0; x < NU; ++x) {
@@ -277,12 +317,14 @@ __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restri
         }
 #pragma unroll
         for (int x = 0; x < NM; ++x) {
-            const int e = t + 256 * x;
-            sm.M[(e / C) * LC + (e % C)] = rm[x];
+            const int e = t + 256 * x, r = e / (C / 4), c4 = (e % (C / 4)) * 4;
+            *reinterpret_cast<float4 *>(&sm.M[r * LC + c4]) = rm[x];
         }
     };
     if (n_chunks > 0) fetch(0);
 
+    const int rp = t >> 3, cq = t & 7;
+    const int r0 = 2 * rp, r1 = r0 + 1;
     for (int chunk = 0; chunk < n_chunks; ++chunk) {
         const int t0 = chunk * C;
         const int n = min(C, L - t0);
@@ -292,57 +334,59 @@ __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restri
         if (chunk + 1 < n_chunks) fetch(chunk + 1);
         __syncthreads();
 
-        // D = U - W S and O = Q S: thread owns rows {2 rp, 2 rp + 1}, cols 4 cq..
-        const int rp = t >> 3, cq = t & 7;
-        const int r0 = 2 * rp, r1 = r0 + 1;
+        // D = U - W S and O = Q S, four d_k indices per step
         float d0[4] = {}, d1[4] = {}, o0[4] = {}, o1[4] = {};
-        for (int i = 0; i < D; ++i) {
-            const float4 s4 = *reinterpret_cast<const float4 *>(&sm.S[i * DVT + 4 * cq]);
-            const float w0 = sm.W[r0 * LD + i], w1 = sm.W[r1 * LD + i];
-            const float q0 = sm.Q[r0 * LD + i], q1 = sm.Q[r1 * LD + i];
-            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                d0[w] = fmaf(w0, sv[w], d0[w]);
-                d1[w] = fmaf(w1, sv[w], d1[w]);
-                o0[w] = fmaf(q0, sv[w], o0[w]);
-                o1[w] = fmaf(q1, sv[w], o1[w]);
-            }
+#pragma unroll 2
+        for (int i = 0; i < D; i += 4) {
+            const float4 w0 = *reinterpret_cast<const float4 *>(&sm.W[r0 * LD + i]);
+            const float4 w1 = *reinterpret_cast<const float4 *>(&sm.W[r1 * LD + i]);
+            const float4 q0 = *reinterpret_cast<const float4 *>(&sm.Q[r0 * LD + i]);
+            const float4 q1 = *reinterpret_cast<const float4 *>(&sm.Q[r1 * LD + i]);
+            const float4 s0 = *reinterpret_cast<const float4 *>(&sm.S[(i + 0) * DVT + 4 * cq]);
+            const float4 s1 = *reinterpret_cast<const float4 *>(&sm.S[(i + 1) * DVT + 4 * cq]);
+            const float4 s2 = *reinterpret_cast<const float4 *>(&sm.S[(i + 2) * DVT + 4 * cq]);
+            const float4 s3 = *reinterpret_cast<const float4 *>(&sm.S[(i + 3) * DVT + 4 * cq]);
+            fma4(d0, w0.x, s0); fma4(d0, w0.y, s1); fma4(d0, w0.z, s2); fma4(d0, w0.w, s3);
+            fma4(d1, w1.x, s0); fma4(d1, w1.y, s1); fma4(d1, w1.z, s2); fma4(d1, w1.w, s3);
+            fma4(o0, q0.x, s0); fma4(o0, q0.y, s1); fma4(o0, q0.z, s2); fma4(o0, q0.w, s3);
+            fma4(o1, q1.x, s0); fma4(o1, q1.y, s1); fma4(o1, q1.z, s2); fma4(o1, q1.w, s3);
         }
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            sm.Dl[r0 * DVT + 4 * cq + w] = sm.U[r0 * DVT + 4 * cq + w] - d0[w];
-            sm.Dl[r1 * DVT + 4 * cq + w] = sm.U[r1 * DVT + 4 * cq + w] - d1[w];
+        {
+            const float4 u0 = *reinterpret_cast<const float4 *>(&sm.U[r0 * DVT + 4 * cq]);
+            const float4 u1 = *reinterpret_cast<const float4 *>(&sm.U[r1 * DVT + 4 * cq]);
+            *reinterpret_cast<float4 *>(&sm.Dl[r0 * DVT + 4 * cq]) =
+                make_float4(u0.x - d0[0], u0.y - d0[1], u0.z - d0[2], u0.w - d0[3]);
+            *reinterpret_cast<float4 *>(&sm.Dl[r1 * DVT + 4 * cq]) =
+                make_float4(u1.x - d1[0], u1.y - d1[1], u1.z - d1[2], u1.w - d1[3]);
         }
         __syncthreads();
 
-        // O += M D (M lower incl. diagonal), write rows < n
-        for (int m = 0; m <= r1; ++m) {
-            const float4 dm = *reinterpret_cast<const float4 *>(&sm.Dl[m * DVT + 4 * cq]);
-            const float dv[4] = {dm.x, dm.y, dm.z, dm.w};
-            const float ma = sm.M[r0 * LC + m], mb = sm.M[r1 * LC + m];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                o0[w] = fmaf(ma, dv[w], o0[w]);
-                o1[w] = fmaf(mb, dv[w], o1[w]);
-            }
+        // O += M D (M lower incl. diagonal, zero above it), write rows < n
+        for (int m = 0; m <= r1; m += 4) {
+            const float4 ma = *reinterpret_cast<const float4 *>(&sm.M[r0 * LC + m]);
+            const float4 mb = *reinterpret_cast<const float4 *>(&sm.M[r1 * LC + m]);
+            const float4 e0 = *reinterpret_cast<const float4 *>(&sm.Dl[(m + 0) * DVT + 4 * cq]);
+            const float4 e1 = *reinterpret_cast<const float4 *>(&sm.Dl[(m + 1) * DVT + 4 * cq]);
+            const float4 e2 = *reinterpret_cast<const float4 *>(&sm.Dl[(m + 2) * DVT + 4 * cq]);
+            const float4 e3 = *reinterpret_cast<const float4 *>(&sm.Dl[(m + 3) * DVT + 4 * cq]);
+            fma4(o0, ma.x, e0); fma4(o0, ma.y, e1); fma4(o0, ma.z, e2); fma4(o0, ma.w, e3);
+            fma4(o1, mb.x, e0); fma4(o1, mb.y, e1); fma4(o1, mb.z, e2); fma4(o1, mb.w, e3);
         }
         if (r0 < n) store4(o + (row0 + r0) * D + j0 + 4 * cq, make_float4(o0[0], o0[1], o0[2], o0[3]));
         if (r1 < n) store4(o + (row0 + r1) * D + j0 + 4 * cq, make_float4(o1[0], o1[1], o1[2], o1[3]));
 
-        // S += K^T D: thread owns rows 4 iq.. (d_k) x cols 4 jq.. (tile)
+        // S += K^T D: thread owns d_k rows 4 iq .. x columns 4 jq .. of the tile
         for (int tile = t; tile < (D / 4) * (DVT / 4); tile += 256) {
             const int iq = tile / (DVT / 4), jq = tile % (DVT / 4);
             float acc[4][4] = {};
+#pragma unroll 4
             for (int m = 0; m < C; ++m) {
+                const float4 km = *reinterpret_cast<const float4 *>(&sm.K[m * LD + 4 * iq]);
                 const float4 dm = *reinterpret_cast<const float4 *>(&sm.Dl[m * DVT + 4 * jq]);
-                const float dv[4] = {dm.x, dm.y, dm.z, dm.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float kk = sm.K[m * LD + 4 * iq + u];
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(kk, dv[w], acc[u][w]);
-                }
+                fma4(acc[0], km.x, dm);
+                fma4(acc[1], km.y, dm);
+                fma4(acc[2], km.z, dm);
+                fma4(acc[3], km.w, dm);
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {

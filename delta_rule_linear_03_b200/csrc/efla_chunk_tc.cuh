@@ -359,6 +359,9 @@ struct SegJob {
     int write_o;      // store the outputs of these chunks
     const float *s0;  // [B*H][d_k][d_v] fp32 (s0_kind 1)
     float *sl;        // final state, [B*H][d_k][d_v] fp32, or null
+    int pair;         // run from zero and from the identity together (no outputs):
+                      // final states to sl (from zero) and sl2 (from the identity)
+    float *sl2;
 };
 constexpr int kMaxJobs = 16;
 // The jobs of one launch (blockIdx.y picks the job) and the sequence's chunk count.
@@ -366,6 +369,220 @@ struct SegPlan {
     int nc, njobs;
     SegJob job[kMaxJobs];
 };
+
+// ---------------------------------------------------------------- paired runs
+// Pass A of the segment-parallel prefill needs, for every middle segment,
+// its final state from zero (S_Z) and from the identity (S_I), and no
+// outputs.  Both runs read the same chunk data, and every state column
+// evolves on its own, so one CTA per (b, h, half of d_v) carries both: its
+// 128 state columns are [S_Z | S_I] over this d_v half.  That is half the
+// CTAs of two separate runs, so twice as many segments fit one wave.  Per
+// chunk (no Q, M or O):
+//   Y  = -W (S_hi + S_lo)                  (tcgen05, M=64 N=128 K=128)
+//   D  = U + Y                             (both halves of the 128 columns)
+//   S += K^T (D_hi + D_lo)                 (tcgen05, M=128 N=128 K=64)
+// Shared memory (offsets from the 1024-byte aligned base):
+//   two stages of W0 W1 K0 K1 U (U: this d_v half, 64 rows x 256 B)
+//   S bf16: hi box 0, hi box 1, lo box 0, lo box 1 (128 rows x 64 columns each)
+//   D bf16: hi box 0, hi box 1, lo box 0, lo box 1 (64 rows x 64 columns each)
+// TMEM: S [0, 128), Y [128, 256).  Y has M = 64: row i sits in lane
+// (i % 16) + 32 (i / 16), so the D read-out uses lanes 0-15 of each warp.
+constexpr uint32_t P2_STAGE = 6 * SLOT;
+constexpr uint32_t P2_SB = 2 * P2_STAGE, P2_DB = P2_SB + 8 * SLOT, P2_BAR = P2_DB + 4 * SLOT;
+static_assert(P2_BAR + 128 + 1024 <= SMEM_BYTES, "paired runs fit the serial kernel's shared memory");
+constexpr uint32_t T2_S = 0, T2_Y = 128, T2_COLS = 256;
+constexpr uint32_t ID2_Y = ptx::idesc_bf16(64, 128, false, true);
+constexpr uint32_t ID2_S = ptx::idesc_bf16(128, 128, true, true);
+enum : int { P2_FULL = 0, P2_EMPTY = 2, P2_SBFULL = 4, P2_DFULL = 5, P2_DELTA = 6, P2_SFULL = 7, P2_DRAIN = 8 };
+
+__device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &tm_k, const unsigned char *ws,
+                                         const SegJob &job, int nc, long bh, int half) {
+    using namespace ptx;
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P2_BAR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + P2_BAR + 96);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P2_BAR + 100);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j0 = half * DVT, cb = job.c0, ncj = job.nch;
+    const unsigned char *img = ws + (size_t)bh * nc * PREP_BYTES;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[P2_FULL + s], 1);
+            mbar_init(&bar[P2_EMPTY + s], 1);
+        }
+        mbar_init(&bar[P2_SBFULL], 256);
+        mbar_init(&bar[P2_DFULL], 1);
+        mbar_init(&bar[P2_DELTA], 256);
+        mbar_init(&bar[P2_SFULL], 1);
+        mbar_init(&bar[P2_DRAIN], 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, T2_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    if (warp < 8) {
+        // ------------------------------------------------------------ TMEM <-> smem warps
+        // Warp w: TMEM lanes 32 (w % 4) .., columns 64 (w / 4) .. + 63 of each
+        // 128-column tile, i.e. the run from zero (w < 4) or from the identity.
+        const int quad = warp & 3, run = warp >> 2;
+        const int row = 32 * quad + lane;           // state row (d_k)
+        const int drow = 16 * quad + (lane & 15);   // chunk row of Y / D (lanes 0-15)
+        const bool dlane = lane < 16;
+        const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
+        float x[32];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {  // initial state: zero, or the identity columns j0 + 32 hh ..
+#pragma unroll
+            for (int c = 0; c < 32; ++c) x[c] = (run == 1 && row == j0 + 32 * hh + c) ? 1.f : 0.f;
+            uint32_t r[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
+            tmem_st32(tl + T2_S + 64 * run + 32 * hh, r);
+            write_split32(sm + P2_SB + run * 2 * SLOT, 4 * SLOT, row, 4 * hh, x);
+        }
+        tmem_st_wait();
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(&bar[P2_SBFULL]);
+        for (int n = 0; n < ncj; ++n) {
+            const int s = n & 1;
+            // D = U + Y for this warp's 64 columns (the same U for both runs)
+            if (!mbar_wait(&bar[P2_DFULL], n & 1, abort_flag)) break;
+            if (!mbar_wait(&bar[P2_FULL + s], (n >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            const unsigned char *urow = sm + s * P2_STAGE + 4 * SLOT + drow * 256;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t r[32];
+                tmem_ld32(tl + T2_Y + 64 * run + 32 * hh, r);
+                tmem_ld_wait(r);
+                if (dlane) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 v =
+                            *reinterpret_cast<const float4 *>(urow + (((uint32_t)(8 * hh + j) ^ (drow & 15)) << 4));
+                        x[4 * j] = v.x + __uint_as_float(r[4 * j]);
+                        x[4 * j + 1] = v.y + __uint_as_float(r[4 * j + 1]);
+                        x[4 * j + 2] = v.z + __uint_as_float(r[4 * j + 2]);
+                        x[4 * j + 3] = v.w + __uint_as_float(r[4 * j + 3]);
+                    }
+                    write_split32(sm + P2_DB + run * SLOT, 2 * SLOT, drow, 4 * hh, x);
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(&bar[P2_DELTA]);
+            // S out of TMEM: the bf16 operand of the next chunk, or the final states
+            if (!mbar_wait(&bar[P2_SFULL], n & 1, abort_flag)) break;
+            tc_fence_after();
+            float *dst = n == ncj - 1 ? (run == 0 ? job.sl : job.sl2) : nullptr;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t r[32];
+                tmem_ld32(tl + T2_S + 64 * run + 32 * hh, r);
+                tmem_ld_wait(r);
+                as_float32(r, x);
+                if (n < ncj - 1) {
+                    write_split32(sm + P2_SB + run * 2 * SLOT, 4 * SLOT, row, 4 * hh, x);
+                } else if (dst) {
+                    float *d = dst + ((size_t)bh * DK + row) * DK + j0 + 32 * hh;
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4)
+                        *reinterpret_cast<float4 *>(d + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+                }
+            }
+            if (n < ncj - 1) {
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(&bar[P2_SBFULL]);
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        const bool leader = lane == 0;
+        for (int n = 0; n < ncj; ++n) {
+            const int s = n & 1;
+            const uint32_t st = sbase + (uint32_t)s * P2_STAGE;
+            if (!warp_wait(&bar[P2_FULL + s], (n >> 1) & 1, abort_flag)) break;
+            if (!warp_wait(&bar[P2_SBFULL], n & 1, abort_flag)) break;
+            tc_fence_after();
+            if (leader) {  // Y = -W (S_hi + S_lo): 8 k-steps over d_k
+                const uint64_t dW = sdesc_sw128(st, 16, 1024);
+                const uint64_t dS = sdesc_sw128(sbase + P2_SB, 2 * SLOT, 1024);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(tmem + T2_Y, dW + (((kk >> 2) * SLOT + (kk & 3) * 32) >> 4),
+                                 dS + ((part * 4 * SLOT + kk * 2048) >> 4), ID2_Y, part | kk);
+                mma_commit(&bar[P2_DFULL]);
+            }
+            __syncwarp();
+            if (!warp_wait(&bar[P2_DELTA], n & 1, abort_flag)) break;
+            tc_fence_after();
+            if (leader) {  // S += K^T (D_hi + D_lo): 4 k-steps over the chunk
+                const uint64_t dKt = sdesc_sw128(st + 2 * SLOT, SLOT, 1024);
+                const uint64_t dD = sdesc_sw128(sbase + P2_DB, SLOT, 1024);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + T2_S, dKt + ((kk * 2048) >> 4), dD + ((part * 2 * SLOT + kk * 2048) >> 4),
+                                 ID2_S, 1);
+                mma_commit(&bar[P2_SFULL]);
+                mma_commit(&bar[P2_EMPTY + s]);
+            }
+            __syncwarp();
+        }
+        __syncwarp();
+        if (leader) mma_commit(&bar[P2_DRAIN]);
+        __syncwarp();
+        int never = 0;
+        mbar_wait(&bar[P2_DRAIN], 0, &never);
+    } else {
+        // ------------------------------------------------------------ loads
+        const bool leader = lane == 0;
+        if (leader) tma_prefetch(&tm_k);
+        int last[2] = {-1, -1};
+        for (int n = 0; n < ncj; ++n) {
+            const int s = n & 1;
+            unsigned char *st = sm + s * P2_STAGE;
+            if (n >= 2 && !warp_wait(&bar[P2_EMPTY + s], ((n >> 1) - 1) & 1, abort_flag)) break;
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            if (leader) {
+                uint64_t *fb = &bar[P2_FULL + s];
+                const unsigned char *src = img + (size_t)(cb + n) * PREP_BYTES;
+                mbar_expect_tx(fb, 6 * SLOT);
+                bulk_load(st, src + IMG_W, SLOT, fb);
+                bulk_load(st + SLOT, src + IMG_W + SLOT, SLOT, fb);
+                tma_load_3d(st + 2 * SLOT, &tm_k, fb, 0, (cb + n) * C, (int)bh);
+                tma_load_3d(st + 3 * SLOT, &tm_k, fb, 64, (cb + n) * C, (int)bh);
+                bulk_load(st + 4 * SLOT, src + IMG_U + half * UHALF, UHALF, fb);
+            }
+            __syncwarp();
+            last[s] = n;
+        }
+        int never = 0;
+        for (int s = 0; s < 2; ++s)
+            if (last[s] >= 0) mbar_wait(&bar[P2_FULL + s], (last[s] >> 1) & 1, &never);
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, T2_COLS);
+    }
+}
 
 template <typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -386,6 +603,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = blockIdx.x % NSPLIT, j0 = half * DVT;
     const SegJob &job = plan.job[blockIdx.y];
     const int nc = plan.nc, cb = job.c0, ncj = job.nch;  // chunks cb .. cb + ncj - 1 of nc
+    if (job.pair) {
+        pair_run(sm, tm_k, ws, job, nc, bh, half);
+        return;
+    }
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -740,7 +961,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
                                                                      const __grid_constant__ CUtensorMap tm_v,
                                                                      const float *__restrict__ beta,
                                                                      unsigned char *__restrict__ ws, int L, int nc,
-                                                                     int euler) {
+                                                                     int c_begin, int c_count, int euler) {
     using namespace ptx;
     extern __shared__ unsigned char psm_raw[];
     unsigned char *sm =
@@ -754,12 +975,13 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_BAR + 48);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + P_BAR + 52);
     const int p = threadIdx.x, w = p >> 5, lane = p & 31;
-    const long gidx = blockIdx.x;
-    // 32-bit quotient and remainder (grid < 2^31; a 64-bit division is a long
-    // instruction sequence on the slow conversion pipe)
-    const unsigned q32 = blockIdx.x / (unsigned)nc;
-    const int chunk = (int)(blockIdx.x - q32 * (unsigned)nc);
+    // chunks c_begin .. c_begin + c_count - 1 of every (b, h); 32-bit quotient
+    // and remainder (grid < 2^31; a 64-bit division is a long instruction
+    // sequence on the slow conversion pipe)
+    const unsigned q32 = blockIdx.x / (unsigned)c_count;
+    const int chunk = c_begin + (int)(blockIdx.x - q32 * (unsigned)c_count);
     const long bh = (long)q32;
+    const long gidx = bh * nc + chunk;
     const int t0 = chunk * C, n = min(C, L - t0);
     const size_t row0 = (size_t)bh * L + t0;
     if (p == 0) EFLA_TR(49, 1023);
@@ -1086,19 +1308,20 @@ inline int sm_count() {
 // The sequence splits into P segments; the state map of segment r is affine,
 // S_out = M_r S_in + S_r, with S_r its final state from zero and M_r its final
 // state from the identity minus S_r.  Pass A runs, in one launch, segment 0
-// from the true S0 (with outputs) and every middle segment from 0 and from I;
-// a chain of small fp32 products then gives every segment's true initial
-// state, S_in(r+1) = M_r S_in(r) + S_r; pass B reruns segments 1..P-1 from
-// those with outputs.  Serial latency drops from nc to about 2 nc / P chunks.
-// P is the largest value in [3, 8] whose pass A (2 CTAs for segment 0, 4 for
-// each middle segment, per (b, h)) fits one wave, with at least
-// kMinSegChunks chunks per segment; otherwise 1 (a single pass).
+// from the true S0 (with outputs) and every middle segment from 0 and from I
+// (both runs in one CTA per d_v half, pair_run); a chain of small fp32
+// products then gives every segment's true initial state,
+// S_in(r+1) = M_r S_in(r) + S_r; pass B reruns segments 1..P-1 from those
+// with outputs.  Serial latency drops from nc to about 2 nc / P chunks.
+// P is the largest value in [3, 8] whose pass A (2 CTAs per segment and
+// (b, h)) fits one wave, with at least kMinSegChunks chunks per segment;
+// otherwise 1 (a single pass).
 constexpr int kMinSegChunks = 16;
 inline int segments(long bh, int nc) {
     const long sms = sm_count();
     int best = 1;
     for (int p = 3; p <= 8; ++p)
-        if (NSPLIT * bh * (1 + 2 * (p - 2)) <= sms && nc / p >= kMinSegChunks) best = p;
+        if (NSPLIT * bh * (p - 1) <= sms && nc / p >= kMinSegChunks) best = p;
     return best;
 }
 inline size_t state_bytes(long bh) { return (size_t)bh * DK * DK * sizeof(float); }
@@ -1161,6 +1384,34 @@ __global__ void __launch_bounds__(256) affine_step_kernel(const float *__restric
         }
 }
 
+// A second stream of the current device and two events, for the part of a
+// segmented prefill's prep that overlaps pass A.  Created on first use, once
+// per device, and kept until the process exits; null if creation failed
+// (the prep then runs on the caller's stream, without the overlap).  Calls
+// that use it are ordered through the events, so calls on different
+// streams stay correct (they share its queue).
+struct SideStream {
+    cudaStream_t s;
+    cudaEvent_t fork, join;
+};
+inline const SideStream *side_stream() {
+    static std::mutex mu;
+    static SideStream made[64];
+    static bool tried[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!tried[dev]) {
+        tried[dev] = true;
+        SideStream x{};
+        if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&
+            cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) == cudaSuccess)
+            made[dev] = x;
+    }
+    return made[dev].join ? &made[dev] : nullptr;
+}
+
 template <typename Tout>
 inline efla_status_t launch(const void *q, const void *k, const void *v, const float *beta, const float *S0,
                             void *o, float *SL, long bh, int L, bool euler, void *ws, cudaStream_t st) {
@@ -1178,10 +1429,29 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     const int nc = (L + C - 1) / C;
     if (grid > 0x7fffffffL || bh * nc > 0x7fffffffL) return EFLA_ERR_SHAPE;
     unsigned char *img = static_cast<unsigned char *>(ws);
-    chunk_prep_tc_kernel<<<(unsigned)(bh * nc), kPrepThreads, P_SMEM, st>>>(mq, mk, mv, beta, img, L, nc,
-                                                                            euler ? 1 : 0);
-    if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
     const int P = segments(bh, nc);
+    auto first = [&](int r) { return (int)((long)r * nc / P); };
+    // With P > 1 the last segment's images are first read by pass B: they are
+    // prepared on a side stream, on the SMs pass A leaves free, after the
+    // rest (the fork waits for that prep, so pass A's CTAs, launched early
+    // as its programmatic dependents, hold their SMs by then).
+    const int split = P > 1 ? first(P - 1) : nc;
+    auto prep = [&](int c_begin, int c_count, cudaStream_t s) {
+        chunk_prep_tc_kernel<<<(unsigned)(bh * c_count), kPrepThreads, P_SMEM, s>>>(mq, mk, mv, beta, img, L, nc,
+                                                                                    c_begin, c_count, euler ? 1 : 0);
+        return cudaGetLastError() == cudaSuccess;
+    };
+    if (!prep(0, split, st)) return EFLA_ERR_CUDA;
+    const SideStream *side = P > 1 ? side_stream() : nullptr;
+    if (P > 1) {
+        if (side) {
+            if (cudaEventRecord(side->fork, st) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess ||
+                !prep(split, nc - split, side->s) || cudaEventRecord(side->join, side->s) != cudaSuccess)
+                return EFLA_ERR_CUDA;
+        } else if (!prep(split, nc - split, st)) {
+            return EFLA_ERR_CUDA;
+        }
+    }
     auto run = [&](const SegPlan &plan) {
         // programmatic stream serialisation: the CTAs may start (and run
         // their prologue) before the previous grid has finished
@@ -1202,7 +1472,7 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     plan.nc = nc;
     if (P == 1) {
         plan.njobs = 1;
-        plan.job[0] = SegJob{0, nc, S0 ? 1 : 0, 1, S0, SL};
+        plan.job[0] = SegJob{0, nc, S0 ? 1 : 0, 1, S0, SL, 0, nullptr};
         return run(plan) ? EFLA_OK : EFLA_ERR_CUDA;
     }
     float *sbuf = reinterpret_cast<float *>(img + (size_t)bh * nc * PREP_BYTES);
@@ -1210,15 +1480,13 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     auto Sin = [&](int r) { return sbuf + (size_t)(r - 1) * sb; };               // r = 1 .. P-1
     auto SZ = [&](int r) { return sbuf + (size_t)(P - 1 + r - 1) * sb; };         // r = 1 .. P-2
     auto SI = [&](int r) { return sbuf + (size_t)(2 * P - 3 + r - 1) * sb; };     // r = 1 .. P-2
-    auto first = [&](int r) { return (int)((long)r * nc / P); };
     // pass A
     plan.njobs = 0;
-    plan.job[plan.njobs++] = SegJob{0, first(1), S0 ? 1 : 0, 1, S0, Sin(1)};
-    for (int r = 1; r <= P - 2; ++r) {
-        plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 0, 0, nullptr, SZ(r)};
-        plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 2, 0, nullptr, SI(r)};
-    }
+    plan.job[plan.njobs++] = SegJob{0, first(1), S0 ? 1 : 0, 1, S0, Sin(1), 0, nullptr};
+    for (int r = 1; r <= P - 2; ++r)
+        plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 0, 0, nullptr, SZ(r), 1, SI(r)};
     if (!run(plan)) return EFLA_ERR_CUDA;
+    if (side && cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess) return EFLA_ERR_CUDA;  // last segment's images
     // the segment chain
     for (int r = 1; r <= P - 2; ++r) {
         affine_step_kernel<DK><<<dim3((unsigned)bh, DK / 32), 256, 0, st>>>(SI(r), SZ(r), Sin(r), Sin(r + 1));
@@ -1227,7 +1495,8 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     // pass B
     plan.njobs = 0;
     for (int r = 1; r <= P - 1; ++r)
-        plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 1, 1, Sin(r), r == P - 1 ? SL : nullptr};
+        plan.job[plan.njobs++] =
+            SegJob{first(r), first(r + 1) - first(r), 1, 1, Sin(r), r == P - 1 ? SL : nullptr, 0, nullptr};
     return run(plan) ? EFLA_OK : EFLA_ERR_CUDA;
 }
 

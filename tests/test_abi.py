@@ -107,8 +107,8 @@ def test_bf16_workspace_includes_segment_states(lib):
     st = 128 * 128 * 4
     # 64 heads, 32 chunks: a single pass
     assert so.efla_chunk_fwd_workspace_size(1, 8, 8, 2048, 128, 128) == 64 * 32 * img
-    # 16 heads, 1024 chunks: P = 3 (pass A needs 2 * 16 * 3 = 96 CTAs)
-    assert so.efla_chunk_fwd_workspace_size(1, 1, 16, 65536, 128, 128) == 16 * 1024 * img + 4 * 16 * st
+    # 16 heads, 1024 chunks: P = 5 (pass A needs 2 CTAs per segment and head: 2 * 16 * 4 = 128)
+    assert so.efla_chunk_fwd_workspace_size(1, 1, 16, 65536, 128, 128) == 16 * 1024 * img + 10 * 16 * st
     # 2 heads, 128 chunks: P = 8 (16 chunks per segment)
     assert so.efla_chunk_fwd_workspace_size(1, 1, 2, 8192, 128, 128) == 2 * 128 * img + 19 * 2 * st
     # too few chunks per segment: a single pass

@@ -5,7 +5,10 @@ With few (b, h) problems the chunk path splits the sequence into P
 segments: pass A runs segment 0 from S0 and every middle segment from zero
 and from the identity, a chain of fp32 products composes the segments'
 affine state maps, pass B reruns segments 1..P-1 from their true initial
-states.  The shapes below select P = 3 (49 chunks) and P = 8 (128 chunks)."""
+states.  A middle segment's two pass-A runs share one CTA per d_v half
+(128 state columns: from zero and from the identity).  The shapes below
+select P = 3 (49 chunks) and P = 8 (128 chunks); the full-size long-context
+test in test_gpu_fullsize.py runs P = 5."""
 import pytest
 import torch
 
