@@ -104,21 +104,16 @@ def decode_bytes(B, H, d, esize, esize_o):
 
 
 def chunk_launches(efla, dtype, B, H, L, d):
-    """Kernel launches of one efla_chunk_fwd: the tensor-core path runs the
-    prep kernel and one serial launch, or, segment-parallel with P segments,
-    the prep, pass A, P - 2 segment-chain steps and pass B (P + 1 in all).
-    P is read off the workspace size (3 P - 5 fp32 states past the per-chunk
-    images); the CUDA-core path runs two kernels."""
-    ws = efla.workspace_size(dtype, B, H, L, d, d)
+    """Kernel launches of one efla_chunk_fwd.  The tensor-core path runs the
+    prep kernel and one serial launch, or, segment-parallel (when the
+    workspace holds segment states past the per-chunk images), five: the
+    prep in two parts (the last segment's on a side stream), pass A, the
+    segment chain and pass B.  The CUDA-core path runs two kernels."""
     if dtype != torch.bfloat16 or d != 128:
         return 2
     nc = (L + 63) // 64
     image = efla.workspace_size(dtype, 1, 1, 64, d, d)  # one chunk's image (never segmented)
-    extra = ws - B * H * nc * image
-    if extra <= 0:
-        return 2
-    P = (extra // (B * H * d * d * 4) + 5) // 3
-    return int(P) + 1
+    return 5 if efla.workspace_size(dtype, B, H, L, d, d) > B * H * nc * image else 2
 
 
 # ------------------------------------------------------------------ clocks

@@ -124,9 +124,17 @@ __device__ long long g_efla_trace[1024 * 64];
     do {                                                                                   \
         if (blockIdx.x == 0) g_efla_trace[((chunk) & 1023) * 64 + ((ev) & 63)] = clock64(); \
     } while (0)
+// the first paired-run job of the launch (blockIdx.y == 1), events 40-47
+#define EFLA_TR2(ev, chunk)                                                                                   \
+    do {                                                                                                      \
+        if (blockIdx.x == 0 && blockIdx.y == 1) g_efla_trace[((chunk) & 1023) * 64 + ((ev) & 63)] = clock64(); \
+    } while (0)
 #else
 #define EFLA_TR(ev, chunk) \
     do {                   \
+    } while (0)
+#define EFLA_TR2(ev, chunk) \
+    do {                    \
     } while (0)
 #endif
 
@@ -378,20 +386,24 @@ struct SegPlan {
 // 128 state columns are [S_Z | S_I] over this d_v half.  That is half the
 // CTAs of two separate runs, so twice as many segments fit one wave.  Per
 // chunk (no Q, M or O):
-//   Y  = -W (S_hi + S_lo)                  (tcgen05, M=64 N=128 K=128)
+//   Y  = [-W; -W] (S_hi + S_lo)            (tcgen05, M=128 N=128 K=128)
 //   D  = U + Y                             (both halves of the 128 columns)
 //   S += K^T (D_hi + D_lo)                 (tcgen05, M=128 N=128 K=64)
+// -W is stacked twice so that every row of Y sits in two TMEM lanes (i and
+// 64 + i): an M = 128 product costs what an M = 64 one does, and all 32
+// lanes of every read-out warp then carry a row (lanes 0-63 the run from
+// zero, lanes 64-127 the run from the identity).
 // Shared memory (offsets from the 1024-byte aligned base):
-//   two stages of W0 W1 K0 K1 U (U: this d_v half, 64 rows x 256 B)
+//   two stages of W0 W0 W1 W1 K0 K1 U (U: this d_v half, 64 rows x 256 B)
 //   S bf16: hi box 0, hi box 1, lo box 0, lo box 1 (128 rows x 64 columns each)
 //   D bf16: hi box 0, hi box 1, lo box 0, lo box 1 (64 rows x 64 columns each)
-// TMEM: S [0, 128), Y [128, 256).  Y has M = 64: row i sits in lane
-// (i % 16) + 32 (i / 16), so the D read-out uses lanes 0-15 of each warp.
-constexpr uint32_t P2_STAGE = 6 * SLOT;
+// TMEM: S [0, 128), Y [128, 256).
+constexpr uint32_t P2_STAGE = 8 * SLOT;
 constexpr uint32_t P2_SB = 2 * P2_STAGE, P2_DB = P2_SB + 8 * SLOT, P2_BAR = P2_DB + 4 * SLOT;
+static_assert(P2_BAR <= OFF_BAR, "paired runs keep their barriers inside the serial kernel's layout");
 static_assert(P2_BAR + 128 + 1024 <= SMEM_BYTES, "paired runs fit the serial kernel's shared memory");
 constexpr uint32_t T2_S = 0, T2_Y = 128, T2_COLS = 256;
-constexpr uint32_t ID2_Y = ptx::idesc_bf16(64, 128, false, true);
+constexpr uint32_t ID2_Y = ptx::idesc_bf16(128, 128, false, true);
 constexpr uint32_t ID2_S = ptx::idesc_bf16(128, 128, true, true);
 enum : int { P2_FULL = 0, P2_EMPTY = 2, P2_SBFULL = 4, P2_DFULL = 5, P2_DELTA = 6, P2_SFULL = 7, P2_DRAIN = 8 };
 
@@ -435,8 +447,11 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
         // 128-column tile, i.e. the run from zero (w < 4) or from the identity.
         const int quad = warp & 3, run = warp >> 2;
         const int row = 32 * quad + lane;           // state row (d_k)
-        const int drow = 16 * quad + (lane & 15);   // chunk row of Y / D (lanes 0-15)
-        const bool dlane = lane < 16;
+        // D read-out: lanes 0-63 hold chunk rows 0-63 for the run from zero,
+        // lanes 64-127 the same rows for the run from the identity; warp w
+        // takes 32 of that run's 64 columns (32 (w / 4) ..)
+        const int drun = quad >> 1, dcol = 32 * (warp >> 2);
+        const int drow = 32 * (quad & 1) + lane;
         const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
         float x[32];
 #pragma unroll
@@ -458,31 +473,31 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             // D = U + Y for this warp's 64 columns (the same U for both runs)
             if (!mbar_wait(&bar[P2_DFULL], n & 1, abort_flag)) break;
             if (!mbar_wait(&bar[P2_FULL + s], (n >> 1) & 1, abort_flag)) break;
+            if (threadIdx.x == 0) EFLA_TR2(41, n);
             tc_fence_after();
-            const unsigned char *urow = sm + s * P2_STAGE + 4 * SLOT + drow * 256;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
+            const unsigned char *urow = sm + s * P2_STAGE + 6 * SLOT + drow * 256;
+            {
                 uint32_t r[32];
-                tmem_ld32(tl + T2_Y + 64 * run + 32 * hh, r);
+                tmem_ld32(tl + T2_Y + 64 * drun + dcol, r);
                 tmem_ld_wait(r);
-                if (dlane) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float4 v =
-                            *reinterpret_cast<const float4 *>(urow + (((uint32_t)(8 * hh + j) ^ (drow & 15)) << 4));
-                        x[4 * j] = v.x + __uint_as_float(r[4 * j]);
-                        x[4 * j + 1] = v.y + __uint_as_float(r[4 * j + 1]);
-                        x[4 * j + 2] = v.z + __uint_as_float(r[4 * j + 2]);
-                        x[4 * j + 3] = v.w + __uint_as_float(r[4 * j + 3]);
-                    }
-                    write_split32(sm + P2_DB + run * SLOT, 2 * SLOT, drow, 4 * hh, x);
+                for (int j = 0; j < 8; ++j) {
+                    const float4 v = *reinterpret_cast<const float4 *>(
+                        urow + (((uint32_t)(dcol / 4 + j) ^ (drow & 15)) << 4));
+                    x[4 * j] = v.x + __uint_as_float(r[4 * j]);
+                    x[4 * j + 1] = v.y + __uint_as_float(r[4 * j + 1]);
+                    x[4 * j + 2] = v.z + __uint_as_float(r[4 * j + 2]);
+                    x[4 * j + 3] = v.w + __uint_as_float(r[4 * j + 3]);
                 }
+                write_split32(sm + P2_DB + drun * SLOT, 2 * SLOT, drow, dcol / 8, x);
             }
             fence_proxy_async();
             tc_fence_before();
             mbar_arrive(&bar[P2_DELTA]);
+            if (threadIdx.x == 0) EFLA_TR2(42, n);
             // S out of TMEM: the bf16 operand of the next chunk, or the final states
             if (!mbar_wait(&bar[P2_SFULL], n & 1, abort_flag)) break;
+            if (threadIdx.x == 0) EFLA_TR2(43, n);
             tc_fence_after();
             float *dst = n == ncj - 1 ? (run == 0 ? job.sl : job.sl2) : nullptr;
 #pragma unroll
@@ -504,6 +519,7 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
                 fence_proxy_async();
                 tc_fence_before();
                 mbar_arrive(&bar[P2_SBFULL]);
+                if (threadIdx.x == 0) EFLA_TR2(44, n);
             }
         }
     } else if (warp == 8) {
@@ -515,6 +531,7 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             if (!warp_wait(&bar[P2_FULL + s], (n >> 1) & 1, abort_flag)) break;
             if (!warp_wait(&bar[P2_SBFULL], n & 1, abort_flag)) break;
             tc_fence_after();
+            if (leader) EFLA_TR2(40, n);
             if (leader) {  // Y = -W (S_hi + S_lo): 8 k-steps over d_k
                 const uint64_t dW = sdesc_sw128(st, 16, 1024);
                 const uint64_t dS = sdesc_sw128(sbase + P2_SB, 2 * SLOT, 1024);
@@ -522,15 +539,16 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tmem + T2_Y, dW + (((kk >> 2) * SLOT + (kk & 3) * 32) >> 4),
+                        mma_bf16(tmem + T2_Y, dW + (((kk >> 2) * 2 * SLOT + (kk & 3) * 32) >> 4),
                                  dS + ((part * 4 * SLOT + kk * 2048) >> 4), ID2_Y, part | kk);
                 mma_commit(&bar[P2_DFULL]);
             }
             __syncwarp();
             if (!warp_wait(&bar[P2_DELTA], n & 1, abort_flag)) break;
             tc_fence_after();
+            if (leader) EFLA_TR2(45, n);
             if (leader) {  // S += K^T (D_hi + D_lo): 4 k-steps over the chunk
-                const uint64_t dKt = sdesc_sw128(st + 2 * SLOT, SLOT, 1024);
+                const uint64_t dKt = sdesc_sw128(st + 4 * SLOT, SLOT, 1024);
                 const uint64_t dD = sdesc_sw128(sbase + P2_DB, SLOT, 1024);
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
@@ -561,12 +579,14 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             if (leader) {
                 uint64_t *fb = &bar[P2_FULL + s];
                 const unsigned char *src = img + (size_t)(cb + n) * PREP_BYTES;
-                mbar_expect_tx(fb, 6 * SLOT);
-                bulk_load(st, src + IMG_W, SLOT, fb);
-                bulk_load(st + SLOT, src + IMG_W + SLOT, SLOT, fb);
-                tma_load_3d(st + 2 * SLOT, &tm_k, fb, 0, (cb + n) * C, (int)bh);
-                tma_load_3d(st + 3 * SLOT, &tm_k, fb, 64, (cb + n) * C, (int)bh);
-                bulk_load(st + 4 * SLOT, src + IMG_U + half * UHALF, UHALF, fb);
+                mbar_expect_tx(fb, 8 * SLOT);
+                bulk_load(st, src + IMG_W, SLOT, fb);  // [-W; -W] for each d_k half
+                bulk_load(st + SLOT, src + IMG_W, SLOT, fb);
+                bulk_load(st + 2 * SLOT, src + IMG_W + SLOT, SLOT, fb);
+                bulk_load(st + 3 * SLOT, src + IMG_W + SLOT, SLOT, fb);
+                tma_load_3d(st + 4 * SLOT, &tm_k, fb, 0, (cb + n) * C, (int)bh);
+                tma_load_3d(st + 5 * SLOT, &tm_k, fb, 64, (cb + n) * C, (int)bh);
+                bulk_load(st + 6 * SLOT, src + IMG_U + half * UHALF, UHALF, fb);
             }
             __syncwarp();
             last[s] = n;
@@ -1317,6 +1337,10 @@ inline int sm_count() {
 // (b, h)) fits one wave, with at least kMinSegChunks chunks per segment;
 // otherwise 1 (a single pass).
 constexpr int kMinSegChunks = 16;
+// The time of a paired-run chunk (pair_run) relative to a single run's, in
+// per cent (clock64 traces of the long-context prefill: 4.45k against 3.78k
+// cycles per chunk).
+constexpr long kPairCost = 118;
 inline int segments(long bh, int nc) {
     const long sms = sm_count();
     int best = 1;
@@ -1412,6 +1436,84 @@ inline const SideStream *side_stream() {
     return made[dev].join ? &made[dev] : nullptr;
 }
 
+// The whole segment chain in one launch: for r = 1 .. steps,
+//   X(r+1) = (SI(r) - SZ(r)) X(r) + SZ(r),
+// with X(1) given and consecutive SI, SZ and X states `stride` floats apart.
+// Column block j of X(r+1) needs only column block j of X(r), so CTA
+// (bh, column block of 32) walks every step on its own, its X block resident
+// in shared memory.  Thread (ty, tx) owns four rows x four columns; the
+// reduction runs in slabs of 32, the next slab of SI - SZ loaded into
+// registers while the current one is used.
+template <int D>
+__global__ void __launch_bounds__(256) affine_chain_kernel(const float *__restrict__ SI, const float *__restrict__ SZ,
+                                                           float *__restrict__ X, int steps, size_t stride) {
+    static_assert(D % 32 == 0 && D <= 128, "D in {32, 64, 128}");
+    constexpr int NS = D / 32;              // slabs per step
+    constexpr int NE = D * 32 / 256;        // slab elements per thread
+    __shared__ float Ms[D][33];
+    __shared__ __align__(16) float Xs[D][36];
+    const size_t base = (size_t)blockIdx.x * D * D;
+    const int cb = 32 * blockIdx.y, tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
+    const bool active = 4 * ty < D;
+    for (int e = tid; e < D * 32; e += 256) {
+        const int r = e >> 5, c = e & 31;
+        Xs[r][c] = X[base + (size_t)r * D + cb + c];
+    }
+    float mreg[NE];
+    auto fetch = [&](int step, int k0) {  // slab k0 of SI(step) - SZ(step)
+        const float *si = SI + (size_t)step * stride + base, *sz = SZ + (size_t)step * stride + base;
+#pragma unroll
+        for (int x = 0; x < NE; ++x) {
+            const int e = tid + 256 * x, r = e >> 5, c = e & 31;
+            const size_t a = (size_t)r * D + k0 + c;
+            mreg[x] = si[a] - sz[a];
+        }
+    };
+    if (steps > 0) fetch(0, 0);
+    for (int step = 0; step < steps; ++step) {
+        float acc[4][4] = {};
+        for (int s = 0; s < NS; ++s) {
+            __syncthreads();  // the previous slab (and, at s = 0, the X block) fully used / written
+#pragma unroll
+            for (int x = 0; x < NE; ++x) {
+                const int e = tid + 256 * x;
+                Ms[e >> 5][e & 31] = mreg[x];
+            }
+            if (s + 1 < NS) fetch(step, 32 * (s + 1));
+            else if (step + 1 < steps) fetch(step + 1, 0);
+            __syncthreads();
+            if (active) {
+#pragma unroll 8
+                for (int k = 0; k < 32; ++k) {
+                    const float4 b = *reinterpret_cast<const float4 *>(&Xs[32 * s + k][4 * tx]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float a = Ms[4 * ty + i][k];
+                        acc[i][0] = fmaf(a, b.x, acc[i][0]);
+                        acc[i][1] = fmaf(a, b.y, acc[i][1]);
+                        acc[i][2] = fmaf(a, b.z, acc[i][2]);
+                        acc[i][3] = fmaf(a, b.w, acc[i][3]);
+                    }
+                }
+            }
+        }
+        __syncthreads();  // every thread is done reading Xs of this step
+        if (active) {
+            const float *sz = SZ + (size_t)step * stride + base;
+            float *out = X + (size_t)(step + 1) * stride + base;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int r = 4 * ty + i, c = 4 * tx + j;
+                    const float y = acc[i][j] + sz[(size_t)r * D + cb + c];
+                    out[(size_t)r * D + cb + c] = y;
+                    Xs[r][c] = y;
+                }
+        }
+    }
+}
+
 template <typename Tout>
 inline efla_status_t launch(const void *q, const void *k, const void *v, const float *beta, const float *S0,
                             void *o, float *SL, long bh, int L, bool euler, void *ws, cudaStream_t st) {
@@ -1430,7 +1532,14 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     if (grid > 0x7fffffffL || bh * nc > 0x7fffffffL) return EFLA_ERR_SHAPE;
     unsigned char *img = static_cast<unsigned char *>(ws);
     const int P = segments(bh, nc);
-    auto first = [&](int r) { return (int)((long)r * nc / P); };
+    // Segment r covers chunks first(r) .. first(r + 1) - 1.  In pass A a
+    // paired-run chunk costs kPairCost (per cent) of a single-run one, so
+    // segment 0 (the only single run of pass A) gets that much more: pass A's
+    // jobs then end together, and segments 1 .. P-1 split the rest evenly.
+    const long seg0 = (long)nc * kPairCost / (kPairCost + 100L * (P - 1));
+    auto first = [&](int r) {
+        return r == 0 ? 0 : (int)(seg0 + (long)(r - 1) * (nc - seg0) / (P - 1));
+    };
     // With P > 1 the last segment's images are first read by pass B: they are
     // prepared on a side stream, on the SMs pass A leaves free, after the
     // rest (the fork waits for that prep, so pass A's CTAs, launched early
@@ -1487,11 +1596,9 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
         plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 0, 0, nullptr, SZ(r), 1, SI(r)};
     if (!run(plan)) return EFLA_ERR_CUDA;
     if (side && cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess) return EFLA_ERR_CUDA;  // last segment's images
-    // the segment chain
-    for (int r = 1; r <= P - 2; ++r) {
-        affine_step_kernel<DK><<<dim3((unsigned)bh, DK / 32), 256, 0, st>>>(SI(r), SZ(r), Sin(r), Sin(r + 1));
-        if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
-    }
+    // the segment chain, one launch: Sin(r + 1) = (SI(r) - SZ(r)) Sin(r) + SZ(r)
+    affine_chain_kernel<DK><<<dim3((unsigned)bh, DK / 32), 256, 0, st>>>(SI(1), SZ(1), Sin(1), P - 2, sb);
+    if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
     // pass B
     plan.njobs = 0;
     for (int r = 1; r <= P - 1; ++r)
