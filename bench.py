@@ -81,6 +81,16 @@ def cpu_model() -> str:
 
 
 # ------------------------------------------------------------------ algorithmic work
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# long-context efla_chunk_fwd call, all launches: an ncu capture of the same
+# call at L = 16384 (16 heads, the same segmented kernels and plan shape)
+# measured 738.6 MB read + 229.3 MB written per call; the per-chunk work and
+# images scale with L, so the full call moves about 4 x 967.9 MB.  It is 3.6 x
+# the algorithmic bytes: the per-chunk workspace image (-W, M, U) makes a
+# round trip, and pass A and pass B both read the middle segments' inputs.
+LONGCTX_TRAFFIC = 4 * 967.9e6
+
+
 def chunk_bytes(B, H, L, d, esize, esize_o, s0: bool, sl: bool = True):
     """HBM bytes of one efla_chunk_fwd that the method itself needs: read q,
     k, v and beta, write o, read S0 (if given) and write S_L once.  With o in
@@ -429,8 +439,10 @@ def run_ours(args):
     flops = chunk_flops(B, H, L, d)
     achieved_tf = flops / (ms_step / 1e3) / 1e12
     roof = hbm_roofline(nbytes, ms_step, peaks, f"efla_chunk_fwd (all {launches_per_step} launches of one call)",
+                        traffic=LONGCTX_TRAFFIC if WORKLOAD == "longctx" else None,
                         note="bytes count o in the q dtype (bf16), 1028 B per head-token; the call writes o "
-                             "in fp32 (the default output dtype, 1284 B per head-token)")
+                             "in fp32 (the default output dtype, 1284 B per head-token). traffic: DRAM bytes "
+                             "of one call, 4 x an ncu capture at L = 16384 (same heads, same kernels)")
     roof["frac_with_fp32_o"] = nbytes_f32o / (ms_step / 1e3) / 1e9 / peaks["hbm"]
 
     line = {
