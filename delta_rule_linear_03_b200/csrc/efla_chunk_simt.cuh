@@ -267,8 +267,9 @@ __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restri
     }
 
     // The tiles of chunk n+1 (W, K, Q, this CTA's U columns, M) are loaded
-    // into registers while chunk n computes, and moved to shared memory at the
-    // top of the next iteration, so no chunk waits on a global-memory round trip.
+    // into registers while chunk n computes its last two products, and moved
+    // to shared memory at the top of the next iteration, so no chunk waits on
+    // a global-memory round trip.
     constexpr int NQ = C * (D / 4) / 256;   // float4s of a C x D tile per thread
     constexpr int NU = C * (DVT / 4) / 256;  // float4s of the C x DVT U tile per thread
     constexpr int NM = C * (C / 4) / 256;    // float4s of the C x C M tile per thread
@@ -331,7 +332,6 @@ __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restri
         const long row0 = bh * (long)L + t0;
         __syncthreads();  // previous chunk's readers are done with the tiles
         stash();
-        if (chunk + 1 < n_chunks) fetch(chunk + 1);
         __syncthreads();
 
         // D = U - W S and O = Q S, four d_k indices per step
@@ -351,6 +351,10 @@ __global__ void __launch_bounds__(256, 1) chunk_state_kernel(const Tin *__restri
             fma4(o0, q0.x, s0); fma4(o0, q0.y, s1); fma4(o0, q0.z, s2); fma4(o0, q0.w, s3);
             fma4(o1, q1.x, s0); fma4(o1, q1.y, s1); fma4(o1, q1.z, s2); fma4(o1, q1.w, s3);
         }
+        // the next chunk's tiles: issued here, so the registers they occupy are
+        // free during the contraction above and the loads land during O += M D
+        // and S += K^T D
+        if (chunk + 1 < n_chunks) fetch(chunk + 1);
         {
             const float4 u0 = *reinterpret_cast<const float4 *>(&sm.U[r0 * DVT + 4 * cq]);
             const float4 u1 = *reinterpret_cast<const float4 *>(&sm.U[r1 * DVT + 4 * cq]);

@@ -124,6 +124,23 @@ __device__ long long g_efla_trace[1024 * 64];
     do {                                                                                   \
         if (blockIdx.x == 0) g_efla_trace[((chunk) & 1023) * 64 + ((ev) & 63)] = clock64(); \
     } while (0)
+// Launch timeline (globaltimer, ns): earliest CTA start and latest CTA end
+// of each launch kind of a call: 0 prep, 1 side-stream prep, 2 pass A,
+// 3 pass B or single pass, 4 segment chain.
+__device__ unsigned long long g_efla_gt[8][2];
+__device__ __forceinline__ unsigned long long efla_gtime() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+#define EFLA_GT_BEGIN(kind) \
+    do {                     \
+        if (threadIdx.x == 0) atomicMin(&g_efla_gt[(kind)][0], efla_gtime()); \
+    } while (0)
+#define EFLA_GT_END(kind)    \
+    do {                     \
+        if (threadIdx.x == 0) atomicMax(&g_efla_gt[(kind)][1], efla_gtime()); \
+    } while (0)
 // the first paired-run job of the launch (blockIdx.y == 1), events 40-47
 #define EFLA_TR2(ev, chunk)                                                                                   \
     do {                                                                                                      \
@@ -135,6 +152,12 @@ __device__ long long g_efla_trace[1024 * 64];
     } while (0)
 #define EFLA_TR2(ev, chunk) \
     do {                    \
+    } while (0)
+#define EFLA_GT_BEGIN(kind) \
+    do {                    \
+    } while (0)
+#define EFLA_GT_END(kind) \
+    do {                  \
     } while (0)
 #endif
 
@@ -623,8 +646,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = blockIdx.x % NSPLIT, j0 = half * DVT;
     const SegJob &job = plan.job[blockIdx.y];
     const int nc = plan.nc, cb = job.c0, ncj = job.nch;  // chunks cb .. cb + ncj - 1 of nc
+    const int gt_kind = (plan.njobs > 1 && plan.job[1].pair) ? 2 : 3;
+    EFLA_GT_BEGIN(gt_kind);
     if (job.pair) {
         pair_run(sm, tm_k, ws, job, nc, bh, half);
+        EFLA_GT_END(gt_kind);
         return;
     }
 
@@ -939,6 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+    EFLA_GT_END(gt_kind);
 }
 
 // ---------------------------------------------------------------- prep kernel
@@ -1002,6 +1029,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     const int chunk = c_begin + (int)(blockIdx.x - q32 * (unsigned)c_count);
     const long bh = (long)q32;
     const long gidx = bh * nc + chunk;
+    EFLA_GT_BEGIN(c_begin == 0 ? 0 : 1);
     const int t0 = chunk * C, n = min(C, L - t0);
     const size_t row0 = (size_t)bh * L + t0;
     if (p == 0) EFLA_TR(49, 1023);
@@ -1271,6 +1299,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
         tc_fence_after();
         tmem_dealloc(tmem, P_TMEM_COLS);
     }
+    EFLA_GT_END(c_begin == 0 ? 0 : 1);
 }
 
 // ---------------------------------------------------------------- host side
@@ -1455,6 +1484,7 @@ __global__ void __launch_bounds__(256) affine_chain_kernel(const float *__restri
     const size_t base = (size_t)blockIdx.x * D * D;
     const int cb = 32 * blockIdx.y, tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
     const bool active = 4 * ty < D;
+    EFLA_GT_BEGIN(4);
     for (int e = tid; e < D * 32; e += 256) {
         const int r = e >> 5, c = e & 31;
         Xs[r][c] = X[base + (size_t)r * D + cb + c];
@@ -1512,6 +1542,7 @@ __global__ void __launch_bounds__(256) affine_chain_kernel(const float *__restri
                 }
         }
     }
+    EFLA_GT_END(4);
 }
 
 template <typename Tout>
