@@ -84,11 +84,11 @@ def cpu_model() -> str:
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
 # long-context efla_chunk_fwd call, all launches: an ncu capture of the same
 # call at L = 16384 (16 heads, the same segmented kernels and plan shape)
-# measured 738.6 MB read + 229.3 MB written per call; the per-chunk work and
-# images scale with L, so the full call moves about 4 x 967.9 MB.  It is 3.6 x
-# the algorithmic bytes: the per-chunk workspace image (-W, M, U) makes a
-# round trip, and pass A and pass B both read the middle segments' inputs.
-LONGCTX_TRAFFIC = 4 * 967.9e6
+# measured 738.5 MB read + 274.9 MB written per call; the per-chunk work and
+# images scale with L, so the full call moves about 4 x 1013.3 MB.  It is
+# 3.8 x the algorithmic bytes: the per-chunk workspace image (-W, M, U)
+# makes a round trip, and pass A and pass B both read the middle segments.
+LONGCTX_TRAFFIC = 4 * 1013.3e6
 
 
 def chunk_bytes(B, H, L, d, esize, esize_o, s0: bool, sl: bool = True):
@@ -116,14 +116,14 @@ def decode_bytes(B, H, d, esize, esize_o):
 def chunk_launches(efla, dtype, B, H, L, d):
     """Kernel launches of one efla_chunk_fwd.  The tensor-core path runs the
     prep kernel and one serial launch, or, segment-parallel (when the
-    workspace holds segment states past the per-chunk images), five: the
-    prep in two parts (the last segment's on a side stream), pass A, the
-    segment chain and pass B.  The CUDA-core path runs two kernels."""
+    workspace holds segment states past the per-chunk images), four: the
+    prep, pass A, the segment chain and pass B.  The CUDA-core path runs two
+    kernels."""
     if dtype != torch.bfloat16 or d != 128:
         return 2
     nc = (L + 63) // 64
     image = efla.workspace_size(dtype, 1, 1, 64, d, d)  # one chunk's image (never segmented)
-    return 5 if efla.workspace_size(dtype, B, H, L, d, d) > B * H * nc * image else 2
+    return 4 if efla.workspace_size(dtype, B, H, L, d, d) > B * H * nc * image else 2
 
 
 # ------------------------------------------------------------------ clocks

@@ -125,8 +125,8 @@ __device__ long long g_efla_trace[1024 * 64];
         if (blockIdx.x == 0) g_efla_trace[((chunk) & 1023) * 64 + ((ev) & 63)] = clock64(); \
     } while (0)
 // Launch timeline (globaltimer, ns): earliest CTA start and latest CTA end
-// of each launch kind of a call: 0 prep, 1 side-stream prep, 2 pass A,
-// 3 pass B or single pass, 4 segment chain.
+// of each launch kind of a call: 0 prep (chunks from 0), 1 prep (a later
+// chunk range), 2 pass A, 3 pass B or single pass, 4 segment chain.
 __device__ unsigned long long g_efla_gt[8][2];
 __device__ __forceinline__ unsigned long long efla_gtime() {
     unsigned long long t;
@@ -1437,34 +1437,6 @@ __global__ void __launch_bounds__(256) affine_step_kernel(const float *__restric
         }
 }
 
-// A second stream of the current device and two events, for the part of a
-// segmented prefill's prep that overlaps pass A.  Created on first use, once
-// per device, and kept until the process exits; null if creation failed
-// (the prep then runs on the caller's stream, without the overlap).  Calls
-// that use it are ordered through the events, so calls on different
-// streams stay correct (they share its queue).
-struct SideStream {
-    cudaStream_t s;
-    cudaEvent_t fork, join;
-};
-inline const SideStream *side_stream() {
-    static std::mutex mu;
-    static SideStream made[64];
-    static bool tried[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!tried[dev]) {
-        tried[dev] = true;
-        SideStream x{};
-        if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) == cudaSuccess &&
-            cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) == cudaSuccess)
-            made[dev] = x;
-    }
-    return made[dev].join ? &made[dev] : nullptr;
-}
-
 // The whole segment chain in one launch: for r = 1 .. steps,
 //   X(r+1) = (SI(r) - SZ(r)) X(r) + SZ(r),
 // with X(1) given and consecutive SI, SZ and X states `stride` floats apart.
@@ -1571,27 +1543,12 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     auto first = [&](int r) {
         return r == 0 ? 0 : (int)(seg0 + (long)(r - 1) * (nc - seg0) / (P - 1));
     };
-    // With P > 1 the last segment's images are first read by pass B: they are
-    // prepared on a side stream, on the SMs pass A leaves free, after the
-    // rest (the fork waits for that prep, so pass A's CTAs, launched early
-    // as its programmatic dependents, hold their SMs by then).
-    const int split = P > 1 ? first(P - 1) : nc;
-    auto prep = [&](int c_begin, int c_count, cudaStream_t s) {
-        chunk_prep_tc_kernel<<<(unsigned)(bh * c_count), kPrepThreads, P_SMEM, s>>>(mq, mk, mv, beta, img, L, nc,
-                                                                                    c_begin, c_count, euler ? 1 : 0);
-        return cudaGetLastError() == cudaSuccess;
-    };
-    if (!prep(0, split, st)) return EFLA_ERR_CUDA;
-    const SideStream *side = P > 1 ? side_stream() : nullptr;
-    if (P > 1) {
-        if (side) {
-            if (cudaEventRecord(side->fork, st) != cudaSuccess || cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess ||
-                !prep(split, nc - split, side->s) || cudaEventRecord(side->join, side->s) != cudaSuccess)
-                return EFLA_ERR_CUDA;
-        } else if (!prep(split, nc - split, st)) {
-            return EFLA_ERR_CUDA;
-        }
-    }
+    // (A variant that prepared the last segment's images on a side stream,
+    // on the SMs pass A leaves free, was measured slower: pass A's serial
+    // chains lost more to the contention than the overlap saved.)
+    chunk_prep_tc_kernel<<<(unsigned)(bh * nc), kPrepThreads, P_SMEM, st>>>(mq, mk, mv, beta, img, L, nc, 0, nc,
+                                                                            euler ? 1 : 0);
+    if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
     auto run = [&](const SegPlan &plan) {
         // programmatic stream serialisation: the CTAs may start (and run
         // their prologue) before the previous grid has finished
@@ -1626,7 +1583,6 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     for (int r = 1; r <= P - 2; ++r)
         plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 0, 0, nullptr, SZ(r), 1, SI(r)};
     if (!run(plan)) return EFLA_ERR_CUDA;
-    if (side && cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess) return EFLA_ERR_CUDA;  // last segment's images
     // the segment chain, one launch: Sin(r + 1) = (SI(r) - SZ(r)) Sin(r) + SZ(r)
     affine_chain_kernel<DK><<<dim3((unsigned)bh, DK / 32), 256, 0, st>>>(SI(1), SZ(1), Sin(1), P - 2, sb);
     if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
