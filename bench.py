@@ -711,38 +711,74 @@ def bench_decode(efla, dev, peaks, with_cpu, reps=3):
 def bench_e2e(efla, dev, x, args, world):
     """The same metric through the public API from pinned host buffers:
     every step copies q, k, v, beta host->device, runs efla_chunk_fwd and
-    copies o and S_L device->host."""
+    copies o and S_L device->host.  Steps are pipelined the way a serving
+    loop would run them: three streams (copy in, compute, copy out) and two
+    device buffer sets, so that step i+1's inputs cross PCIe while step i
+    computes and step i-1's outputs come back (PCIe is full duplex).  Each
+    step still moves all of its own inputs and outputs inside the timed
+    region; a buffer set is refilled only after the step that used it has
+    been copied out."""
     hq, hk, hv, hb = (x[n].pin_memory() for n in ("q", "k", "v", "beta"))
     B, H, L, d = hq.shape
-    ho = torch.empty(B, H, L, d, dtype=torch.float32).pin_memory()
-    hS = torch.empty(B, H, d, d, dtype=torch.float32).pin_memory()
-    dq, dk, dv, db = (torch.empty_like(t, device=dev) for t in (hq, hk, hv, hb))
-    do = torch.empty(B, H, L, d, dtype=torch.float32, device=dev)
-    dS = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    ho = [torch.empty(B, H, L, d, dtype=torch.float32).pin_memory() for _ in range(2)]
+    hS = [torch.empty(B, H, d, d, dtype=torch.float32).pin_memory() for _ in range(2)]
+    din = [tuple(torch.empty_like(t, device=dev) for t in (hq, hk, hv, hb)) for _ in range(2)]
+    do = [torch.empty(B, H, L, d, dtype=torch.float32, device=dev) for _ in range(2)]
+    dS = [torch.empty(B, H, d, d, dtype=torch.float32, device=dev) for _ in range(2)]
+    ws = torch.empty(max(efla.workspace_size(hq.dtype, B, H, L, d, d), 16), dtype=torch.uint8, device=dev)
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
-    def step():
-        for dst, src in ((dq, hq), (dk, hk), (dv, hv), (db, hb)):
-            dst.copy_(src, non_blocking=True)
-        efla.chunk_fwd(dq, dk, dv, db, None, o=do, S_L=dS)
-        ho.copy_(do, non_blocking=True)
-        hS.copy_(dS, non_blocking=True)
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_comp[b])       # step i-2 has finished reading this input set
+            for dst, src in zip(din[b], (hq, hk, hv, hb)):
+                dst.copy_(src, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[b])
+            s_comp.wait_event(ev_out[b])      # step i-2's outputs have left this output set
+            efla.chunk_fwd(*din[b], None, o=do[b], S_L=dS[b], workspace=ws)
+            ev_comp[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            ho[b].copy_(do[b], non_blocking=True)
+            hS[b].copy_(dS[b], non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(3):
-        step()
+    def run(n):
+        cur = torch.cuda.current_stream(dev)
+        for s in (s_in, s_comp, s_out):
+            s.wait_stream(cur)
+        for i in range(n):
+            step(i)
+        for s in (s_in, s_comp, s_out):
+            cur.wait_stream(s)
+
+    run(3)
     torch.cuda.synchronize()
     n = max(3, min(args.steps, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     e0.record()
-    for _ in range(n):
-        step()
+    run(n)
     e1.record()
     torch.cuda.synchronize()
+    if efla.last_error() != 0:
+        raise RuntimeError("efla_chunk_fwd reported a device-side error")
     ms = max_over_ranks(e0.elapsed_time(e1), world)
+    barrier(world)
+    e0.record()
+    run(1)                                     # one step alone: its latency, copies included
+    e1.record()
+    torch.cuda.synchronize()
+    one_ms = max_over_ranks(e0.elapsed_time(e1), world)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb))
-    d2h = ho.numel() * ho.element_size() + hS.numel() * hS.element_size()
+    d2h = ho[0].numel() * ho[0].element_size() + hS[0].numel() * hS[0].element_size()
     return {"value": world * B * L * n / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": n}
+            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n, "single_step_ms": one_ms,
+            "pipeline": "3 streams (copy in / compute / copy out), 2 buffer sets; steps overlap"}
 
 
 def run_profile_case(case: str, calls: int, seq_len=None):

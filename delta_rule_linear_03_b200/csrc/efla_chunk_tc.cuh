@@ -18,15 +18,22 @@
 //                                                      T' as bf16 hi + lo)
 //   -> workspace: -W (bf16), M (bf16), U (fp32)
 //   kernel chunk_tc_kernel, serial over the chunks of one (b, h, d_v half):
-//   Y  = [Q; -W] S          ->  [Q S; -W S]           (tcgen05, M=128 N=64 K=128)
+//   Y  = [Q; -W] S          ->  [Q S; -W S]           (tcgen05, M=128 N=128 K=128)
 //   D  = U + (-W S)                                   (CUDA cores, TMEM -> smem)
-//   S += K^T D                                        (tcgen05, N=64 K=64)
-//   Y += [M; *] D           ->  O = Q S + M D         (tcgen05, N=64 K=64)
+//   S += K^T D                                        (tcgen05, M=128 N=128 K=64)
+//   Y += [M; *] D           ->  O = Q S + M D         (tcgen05, M=128 N=128 K=64)
 //
 // Every product is stacked to M = 128 rows so the accumulator of each
 // tcgen05.mma occupies all 128 TMEM lanes, one row per lane.  (In the last
 // product the lower 64 rows of the A operand are whatever follows M in shared
 // memory: they only add into the -W S rows of Y, which are dead by then.)
+// The hi and lo halves of a split operand sit side by side as one N = 128
+// operand, [S_hi | S_lo] and [D_hi | D_lo], so each product is half as many
+// tcgen05.mma ops as with the halves issued one after the other (an N = 128
+// op costs about a third more than an N = 64 one; an M = 64 op costs what an
+// M = 128 op does).  The two 64-column halves of each accumulator are summed
+// when read out; the state is kept as S = S_a + S_b, two fp32 accumulators
+// that collect K^T D_hi and K^T D_lo.
 //
 // Precision: q, k, v are exact bf16 operands.  S, D and T' are fp32 values
 // fed to the bf16 tensor cores as a hi + lo pair of bf16 (x = hi + lo to ~16
@@ -90,9 +97,10 @@ constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
-// TMEM columns (fp32, 128 lanes): the state tile, then two Y accumulators
-// (by chunk parity) so O of chunk n can wait in TMEM while Y(n+1) runs.
-constexpr uint32_t T_S = 0, T_Y = 64, TMEM_COLS = 256;
+// TMEM columns (fp32, 128 lanes): the state tile [S_a | S_b], then two Y
+// accumulators [Y S_hi | Y S_lo] (by chunk parity) so O of chunk n can wait
+// in TMEM while Y(n+1) runs.
+constexpr uint32_t T_S = 0, T_Y = 128, TMEM_COLS = 512;
 
 enum : int {
     B_FULLA = 0,    // [2] stage part A landed (TMA transaction count)
@@ -111,8 +119,8 @@ enum : int {
 // come in pairs indexed by chunk parity: each then completes once per two
 // chunks, so a parity wait can never see it two phases ahead.
 
-constexpr uint32_t ID_Y = ptx::idesc_bf16(128, 64, false, true);
-constexpr uint32_t ID_S = ptx::idesc_bf16(128, 64, true, true);
+constexpr uint32_t ID_Y = ptx::idesc_bf16(128, 128, false, true);
+constexpr uint32_t ID_S = ptx::idesc_bf16(128, 128, true, true);
 
 // Optional timeline trace (compile with -DEFLA_TRACE): threads of CTA 0
 // store clock64() at their hand-off points into fixed slots
@@ -710,7 +718,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t r[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
-            tmem_st32(tl + T_S + c0, r);
+            tmem_st32(tl + T_S + c0, r);  // S_a = S0
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = 0u;
+            tmem_st32(tl + T_S + 64 + c0, r);  // S_b = 0
             tmem_st_wait();
             write_split32(sm + OFF_SB, 2 * SLOT, row, 4 * cpart, x);
             fence_proxy_async();
@@ -724,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // sets the abort flag, which makes every other wait give up at once.
         for (int n = 0; n < ncj; ++n) {
             const int b = n & 1;
-            const uint32_t ty = T_Y + 64 * b + c0;
+            const uint32_t ty = T_Y + 128 * b + c0;
             if (dwarp) {
                 // D = U + (-W S): TMEM lanes 64..127 of Y, plus U from the stage
                 const int c = row - 64;
@@ -735,8 +746,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(&bar[B_FULLB + b], (n >> 1) & 1, abort_flag)) break;
                 if (row == 64 && cpart == 0) EFLA_TR(10, n);
                 tc_fence_after();
-                uint32_t r[32];
-                tmem_ld32(tl + ty, r);
+                uint32_t r[32], r2[32];
+                tmem_ld32(tl + ty, r);        // -W S_hi
+                tmem_ld32(tl + ty + 64, r2);  // -W S_lo
                 const unsigned char *urow = sm + b * STAGE + SL_U * SLOT + c * 256;
                 float u[32];
 #pragma unroll
@@ -749,8 +761,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     u[4 * j + 3] = v.w;
                 }
                 tmem_ld_wait(r);
+                tmem_ld_wait(r2);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = u[i] + __uint_as_float(r[i]);
+                for (int i = 0; i < 32; ++i) x[i] = u[i] + (__uint_as_float(r[i]) + __uint_as_float(r2[i]));
                 write_split32(sm + OFF_DB + b * 2 * SLOT, SLOT, c, 4 * cpart, x);
                 fence_proxy_async();
                 tc_fence_before();
@@ -762,11 +775,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok && dwarp) break;
             if (ok) {
                 tc_fence_after();
-                uint32_t r[32];
-                tmem_ld32(tl + T_S + c0, r);
+                uint32_t r[32], r2[32];
+                tmem_ld32(tl + T_S + c0, r);        // S_a
+                tmem_ld32(tl + T_S + 64 + c0, r2);  // S_b
                 tmem_ld_wait(r);
+                tmem_ld_wait(r2);
                 if (row == 64 && cpart == 0) EFLA_TR(30, n);
-                as_float32(r, x);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
                 write_split32(sm + OFF_SB, 2 * SLOT, row, 4 * cpart, x);
                 if (row == 64 && cpart == 0) EFLA_TR(31, n);
                 fence_proxy_async();
@@ -790,11 +806,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (bar_any(3, 128, !okO || *abort_flag)) break;
                 {
                     tc_fence_after();
-                    uint32_t r[32];
-                    tmem_ld32(tl + ty, r);
+                    uint32_t r[32], r2[32];
+                    tmem_ld32(tl + ty, r);        // Q S_hi + M D_hi
+                    tmem_ld32(tl + ty + 64, r2);  // Q S_lo + M D_lo
                     tmem_ld_wait(r);
+                    tmem_ld_wait(r2);
                     tc_fence_before();
                     mbar_arrive(&bar[B_OREAD + b]);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
                     if (row == 0 && cpart == 0) EFLA_TR(14, n);
                     // staging: 128-byte-swizzled boxes of 128-byte rows -- fp32: two
                     // 32-column boxes (one per column half c0); bf16: one 64-column box
@@ -836,7 +856,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // builds its base descriptors once; the unrolled k-steps add
         // compile-time offsets, keeping the issuing lane ahead of the pipe.
         const bool leader = lane == 0;
-        const uint64_t dSB = sdesc_sw128(sbase + OFF_SB, SLOT, 1024);
+        // N = 128 operands [S_hi | S_lo] (the lo tile 16 KB after hi) and
+        // [D_hi | D_lo] (8 KB apart): the leading byte offset of the
+        // MN-major descriptor steps from the first 64 columns to the second.
+        const uint64_t dSB = sdesc_sw128(sbase + OFF_SB, 2 * SLOT, 1024);
         const uint64_t dDB = sdesc_sw128(sbase + OFF_DB, SLOT, 1024);
         // O += M (D_hi + D_lo) of chunk m: issued behind Y of chunk m+1, so it
         // runs while the state warps convert D of chunk m+1 (its readers then
@@ -846,17 +869,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dM = sdesc_sw128(sbase + (uint32_t)b * STAGE + SL_M * SLOT, 16, 1024);
             const uint64_t dD = dDB + ((b * 2 * SLOT) >> 4);
 #pragma unroll
-            for (int part = 0; part < 2; ++part)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + T_Y + 64 * b, dM + ((kk * 32) >> 4), dD + ((part * SLOT + kk * 2048) >> 4), ID_Y, 1);
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tmem + T_Y + 128 * b, dM + ((kk * 32) >> 4), dD + ((kk * 2048) >> 4), ID_Y, 1);
             mma_commit(&bar[B_OFULL + b]);
             mma_commit(&bar[B_EMPTYB + b]);
         };
         int n = 0;
         for (; n < ncj; ++n) {
             const int s = n & 1;
-            const uint32_t sa = sbase + (uint32_t)s * STAGE, ty = tmem + T_Y + 64 * s;
+            const uint32_t sa = sbase + (uint32_t)s * STAGE, ty = tmem + T_Y + 128 * s;
             // Y = [Q; -W] (S_hi + S_lo) after: part A of the stage landed, O of
             // chunk n-2 left this Y buffer (both long done: waited while the
             // state warps still convert S), the bf16 state of chunk n written.
@@ -869,11 +890,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 EFLA_TR(20, n);
                 const uint64_t dA = sdesc_sw128(sa + SL_Q0 * SLOT, 16, 1024);
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(ty, dA + (((kk >> 2) * 2 * SLOT + (kk & 3) * 32) >> 4),
-                                 dSB + ((part * 2 * SLOT + kk * 2048) >> 4), ID_Y, part | kk);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(ty, dA + (((kk >> 2) * 2 * SLOT + (kk & 3) * 32) >> 4), dSB + ((kk * 2048) >> 4), ID_Y,
+                             kk);
                 mma_commit(&bar[B_DFULL]);
                 mma_commit(&bar[B_EMPTYA + s]);
                 EFLA_TR(24, n);
@@ -889,10 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t dKt = sdesc_sw128(sa + SL_K0 * SLOT, SLOT, 1024);
                 const uint64_t dD = dDB + ((s * 2 * SLOT) >> 4);
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + T_S, dKt + ((kk * 2048) >> 4), dD + ((part * SLOT + kk * 2048) >> 4), ID_S, 1);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + T_S, dKt + ((kk * 2048) >> 4), dD + ((kk * 2048) >> 4), ID_S, 1);
                 mma_commit(&bar[B_SFULL]);
                 EFLA_TR(25, n);
             }
