@@ -417,9 +417,9 @@ struct SegPlan {
 // 128 state columns are [S_Z | S_I] over this d_v half.  That is half the
 // CTAs of two separate runs, so twice as many segments fit one wave.  Per
 // chunk (no Q, M or O):
-//   Y  = [-W; -W] (S_hi + S_lo)            (tcgen05, M=128 N=128 K=128)
-//   D  = U + Y                             (both halves of the 128 columns)
-//   S += K^T (D_hi + D_lo)                 (tcgen05, M=128 N=128 K=64)
+//   Y  = [-W; -W] [S_hi | S_lo]            (tcgen05, M=128 N=256 K=128)
+//   D  = U + Y_hi + Y_lo                   (both halves of the 128 columns)
+//   S += K^T [D_hi | D_lo]                 (tcgen05, M=128 N=256 K=64)
 // -W is stacked twice so that every row of Y sits in two TMEM lanes (i and
 // 64 + i): an M = 128 product costs what an M = 64 one does, and all 32
 // lanes of every read-out warp then carry a row (lanes 0-63 the run from
@@ -428,14 +428,18 @@ struct SegPlan {
 //   two stages of W0 W0 W1 W1 K0 K1 U (U: this d_v half, 64 rows x 256 B)
 //   S bf16: hi box 0, hi box 1, lo box 0, lo box 1 (128 rows x 64 columns each)
 //   D bf16: hi box 0, hi box 1, lo box 0, lo box 1 (64 rows x 64 columns each)
-// TMEM: S [0, 128), Y [128, 256).
+// The hi and lo halves of S and D sit side by side as one N = 256 operand
+// (as in the single run): the state is S_a + S_b, and Y is read out as
+// Y_hi + Y_lo.
+// TMEM: S [0, 256) = [S_a | S_b], Y [256, 512) = [Y_hi | Y_lo], each half
+// 128 columns [run from zero | run from the identity].
 constexpr uint32_t P2_STAGE = 8 * SLOT;
 constexpr uint32_t P2_SB = 2 * P2_STAGE, P2_DB = P2_SB + 8 * SLOT, P2_BAR = P2_DB + 4 * SLOT;
 static_assert(P2_BAR <= OFF_BAR, "paired runs keep their barriers inside the serial kernel's layout");
 static_assert(P2_BAR + 128 + 1024 <= SMEM_BYTES, "paired runs fit the serial kernel's shared memory");
-constexpr uint32_t T2_S = 0, T2_Y = 128, T2_COLS = 256;
-constexpr uint32_t ID2_Y = ptx::idesc_bf16(128, 128, false, true);
-constexpr uint32_t ID2_S = ptx::idesc_bf16(128, 128, true, true);
+constexpr uint32_t T2_S = 0, T2_Y = 256, T2_COLS = 512;
+constexpr uint32_t ID2_Y = ptx::idesc_bf16(128, 256, false, true);
+constexpr uint32_t ID2_S = ptx::idesc_bf16(128, 256, true, true);
 enum : int { P2_FULL = 0, P2_EMPTY = 2, P2_SBFULL = 4, P2_DFULL = 5, P2_DELTA = 6, P2_SFULL = 7, P2_DRAIN = 8 };
 
 __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &tm_k, const unsigned char *ws,
@@ -493,6 +497,9 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
             tmem_st32(tl + T2_S + 64 * run + 32 * hh, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = 0u;
+            tmem_st32(tl + T2_S + 128 + 64 * run + 32 * hh, r);
             write_split32(sm + P2_SB + run * 2 * SLOT, 4 * SLOT, row, 4 * hh, x);
         }
         tmem_st_wait();
@@ -508,17 +515,19 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             tc_fence_after();
             const unsigned char *urow = sm + s * P2_STAGE + 6 * SLOT + drow * 256;
             {
-                uint32_t r[32];
-                tmem_ld32(tl + T2_Y + 64 * drun + dcol, r);
+                uint32_t r[32], r2[32];
+                tmem_ld32(tl + T2_Y + 64 * drun + dcol, r);         // Y_hi
+                tmem_ld32(tl + T2_Y + 128 + 64 * drun + dcol, r2);  // Y_lo
                 tmem_ld_wait(r);
+                tmem_ld_wait(r2);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float4 v = *reinterpret_cast<const float4 *>(
                         urow + (((uint32_t)(dcol / 4 + j) ^ (drow & 15)) << 4));
-                    x[4 * j] = v.x + __uint_as_float(r[4 * j]);
-                    x[4 * j + 1] = v.y + __uint_as_float(r[4 * j + 1]);
-                    x[4 * j + 2] = v.z + __uint_as_float(r[4 * j + 2]);
-                    x[4 * j + 3] = v.w + __uint_as_float(r[4 * j + 3]);
+                    x[4 * j] = v.x + (__uint_as_float(r[4 * j]) + __uint_as_float(r2[4 * j]));
+                    x[4 * j + 1] = v.y + (__uint_as_float(r[4 * j + 1]) + __uint_as_float(r2[4 * j + 1]));
+                    x[4 * j + 2] = v.z + (__uint_as_float(r[4 * j + 2]) + __uint_as_float(r2[4 * j + 2]));
+                    x[4 * j + 3] = v.w + (__uint_as_float(r[4 * j + 3]) + __uint_as_float(r2[4 * j + 3]));
                 }
                 write_split32(sm + P2_DB + drun * SLOT, 2 * SLOT, drow, dcol / 8, x);
             }
@@ -533,10 +542,13 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             float *dst = n == ncj - 1 ? (run == 0 ? job.sl : job.sl2) : nullptr;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                uint32_t r[32];
-                tmem_ld32(tl + T2_S + 64 * run + 32 * hh, r);
+                uint32_t r[32], r2[32];
+                tmem_ld32(tl + T2_S + 64 * run + 32 * hh, r);         // S_a
+                tmem_ld32(tl + T2_S + 128 + 64 * run + 32 * hh, r2);  // S_b
                 tmem_ld_wait(r);
-                as_float32(r, x);
+                tmem_ld_wait(r2);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
                 if (n < ncj - 1) {
                     write_split32(sm + P2_SB + run * 2 * SLOT, 4 * SLOT, row, 4 * hh, x);
                 } else if (dst) {
@@ -563,30 +575,25 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             if (!warp_wait(&bar[P2_SBFULL], n & 1, abort_flag)) break;
             tc_fence_after();
             if (leader) EFLA_TR2(40, n);
-            if (leader) {  // Y = -W (S_hi + S_lo): 8 k-steps over d_k
+            if (leader) {  // Y = -W [S_hi | S_lo]: 8 k-steps over d_k
                 const uint64_t dW = sdesc_sw128(st, 16, 1024);
                 const uint64_t dS = sdesc_sw128(sbase + P2_SB, 2 * SLOT, 1024);
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tmem + T2_Y, dW + (((kk >> 2) * 2 * SLOT + (kk & 3) * 32) >> 4),
-                                 dS + ((part * 4 * SLOT + kk * 2048) >> 4), ID2_Y, part | kk);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem + T2_Y, dW + (((kk >> 2) * 2 * SLOT + (kk & 3) * 32) >> 4),
+                             dS + ((kk * 2048) >> 4), ID2_Y, kk);
                 mma_commit(&bar[P2_DFULL]);
             }
             __syncwarp();
             if (!warp_wait(&bar[P2_DELTA], n & 1, abort_flag)) break;
             tc_fence_after();
             if (leader) EFLA_TR2(45, n);
-            if (leader) {  // S += K^T (D_hi + D_lo): 4 k-steps over the chunk
+            if (leader) {  // S += K^T [D_hi | D_lo]: 4 k-steps over the chunk
                 const uint64_t dKt = sdesc_sw128(st + 4 * SLOT, SLOT, 1024);
                 const uint64_t dD = sdesc_sw128(sbase + P2_DB, SLOT, 1024);
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + T2_S, dKt + ((kk * 2048) >> 4), dD + ((part * 2 * SLOT + kk * 2048) >> 4),
-                                 ID2_S, 1);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + T2_S, dKt + ((kk * 2048) >> 4), dD + ((kk * 2048) >> 4), ID2_S, 1);
                 mma_commit(&bar[P2_SFULL]);
                 mma_commit(&bar[P2_EMPTY + s]);
             }
@@ -741,10 +748,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c = row - 64;
                 // (the stage's own barrier too: U landed by the bulk copy is
                 // visible to the threads that observe that barrier's phase)
+                if (!mbar_wait(&bar[B_FULLB + b], (n >> 1) & 1, abort_flag)) break;
                 if (!mbar_wait(&bar[B_DFULL], n & 1, abort_flag)) break;
                 if (row == 64 && cpart == 0) EFLA_TR(28, n);
-                if (!mbar_wait(&bar[B_FULLB + b], (n >> 1) & 1, abort_flag)) break;
-                if (row == 64 && cpart == 0) EFLA_TR(10, n);
                 tc_fence_after();
                 uint32_t r[32], r2[32];
                 tmem_ld32(tl + ty, r);        // -W S_hi
@@ -1111,6 +1117,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
         if (h == 0) alpha[r] = (r < n) ? gate_alpha(beta_r, ss, euler != 0) : 0.f;
     }
     ok = ok && wait_all(2, 0);  // (also publishes alpha)
+    if (p == 0) EFLA_TR(40, 1023);
     tc_fence_after();
     unsigned char *out = ws + (size_t)gidx * PREP_BYTES;
     const int quad = w & 3, cpart = w >> 2;
@@ -1235,6 +1242,7 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
     const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16) + 64 * cpart;
     if (p == 0 && ok) issue_wu(0, 3);
     ok = ok && wait_all(3, 0);
+    if (p == 0) EFLA_TR(41, 1023);
     tc_fence_after();
     if (ok) {
 #pragma unroll
@@ -1264,8 +1272,10 @@ __global__ void __launch_bounds__(kPrepThreads, 4) chunk_prep_tc_kernel(const __
         bulk_store(out + IMG_W + SLOT, sm + P_KQ + 2 * SLOT, SLOT);
         bulk_commit();
         issue_wu(SLOT, 4);
+        EFLA_TR(42, 1023);
     }
     ok = ok && wait_all(4, 0);
+    if (p == 0) EFLA_TR(43, 1023);
     tc_fence_after();
     if (ok) {
 #pragma unroll
@@ -1384,9 +1394,9 @@ inline int sm_count() {
 // otherwise 1 (a single pass).
 constexpr int kMinSegChunks = 16;
 // The time of a paired-run chunk (pair_run) relative to a single run's, in
-// per cent (clock64 traces of the long-context prefill: 4.45k against 3.78k
-// cycles per chunk).
-constexpr long kPairCost = 118;
+// per cent (clock64 traces: 4.45k cycles per paired-run chunk on the
+// long-context prefill against 3.28k per single-run chunk on lm340m).
+constexpr long kPairCost = 136;
 inline int segments(long bh, int nc) {
     const long sms = sm_count();
     int best = 1;
