@@ -149,6 +149,13 @@ __device__ __forceinline__ unsigned long long efla_gtime() {
     do {                     \
         if (threadIdx.x == 0) atomicMax(&g_efla_gt[(kind)][1], efla_gtime()); \
     } while (0)
+// Per-CTA times of the serial kernel (globaltimer, ns): [launch kind - 2]
+// [job][CTA][0: past the grid dependency, 1: end]
+__device__ unsigned long long g_efla_cta[2][16][64][2];
+#define EFLA_CTA(kind, i)                                                                         \
+    do {                                                                                        \
+        if (threadIdx.x == 0 && blockIdx.x < 64) g_efla_cta[(kind) - 2][blockIdx.y][blockIdx.x][i] = efla_gtime(); \
+    } while (0)
 // the first paired-run job of the launch (blockIdx.y == 1), events 40-47
 #define EFLA_TR2(ev, chunk)                                                                                   \
     do {                                                                                                      \
@@ -165,6 +172,9 @@ __device__ __forceinline__ unsigned long long efla_gtime() {
     do {                    \
     } while (0)
 #define EFLA_GT_END(kind) \
+    do {                  \
+    } while (0)
+#define EFLA_CTA(kind, i) \
     do {                  \
     } while (0)
 #endif
@@ -475,6 +485,7 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    EFLA_CTA(2, 0);
 
     if (warp < 8) {
         // ------------------------------------------------------------ TMEM <-> smem warps
@@ -665,6 +676,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     EFLA_GT_BEGIN(gt_kind);
     if (job.pair) {
         pair_run(sm, tm_k, ws, job, nc, bh, half);
+        EFLA_CTA(gt_kind, 1);
         EFLA_GT_END(gt_kind);
         return;
     }
@@ -698,6 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // kernel, or the segment chain): the prologue above overlaps that grid's
     // last wave; nothing it wrote is read before this wait returns.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    EFLA_CTA(gt_kind, 0);
 
     if (warp < 8) {
         // ------------------------------------------------------------ TMEM <-> smem warps
@@ -988,6 +1001,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+    EFLA_CTA(gt_kind, 1);
     EFLA_GT_END(gt_kind);
 }
 
