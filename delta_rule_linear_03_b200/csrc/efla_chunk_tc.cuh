@@ -107,12 +107,12 @@ enum : int {
     B_FULLB = 2,    // [2] stage part B landed
     B_EMPTYA = 4,   // [2] part A free again (commit after Y)
     B_EMPTYB = 6,   // [2] part B free again (commit after O)
-    B_SBFULL = 8,   // bf16 S tile written (256 threads)
+    B_SBFULL = 8,   // bf16 S tile written (8 warps)
     B_DFULL = 9,    // Y = [Q; -W] S done
-    B_DELTA = 10,   // bf16 D written (128 threads)
+    B_DELTA = 10,   // bf16 D written (4 warps)
     B_SFULL = 11,   // S += K^T D done
     B_DRAIN = 12,   // final drain of the MMA pipe
-    B_OREAD = 13,   // [2] O of a chunk read out of Y buffer b (128 threads)
+    B_OREAD = 13,   // [2] O of a chunk read out of Y buffer b (4 warps)
     B_OFULL = 15,   // [2] O += M D done for Y buffer b
 };
 // Barriers that complete once per chunk but can be waited on a chunk late
@@ -400,6 +400,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort));
 }
 
+// One arrival per warp (barriers counted in warps): every lane has finished
+// its shared-memory writes (and fenced them for the async proxy) and its
+// TMEM loads; the warp synchronises, then lane 0 arrives.  One arrival
+// instead of 32 keeps the barrier's last arrival, the one the waiting MMA
+// thread is woken by, from queueing behind the warp's other 31.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) ptx::mbar_arrive(bar);
+}
+
 // One run of the serial kernel over a contiguous range of chunks, for every
 // (b, h, d_v half) of the grid: the whole sequence, or one segment of it.
 struct SegJob {
@@ -469,9 +479,9 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             mbar_init(&bar[P2_FULL + s], 1);
             mbar_init(&bar[P2_EMPTY + s], 1);
         }
-        mbar_init(&bar[P2_SBFULL], 256);
+        mbar_init(&bar[P2_SBFULL], 8);  // one arrival per converter warp
         mbar_init(&bar[P2_DFULL], 1);
-        mbar_init(&bar[P2_DELTA], 256);
+        mbar_init(&bar[P2_DELTA], 8);
         mbar_init(&bar[P2_SFULL], 1);
         mbar_init(&bar[P2_DRAIN], 1);
         fence_mbar_init();
@@ -516,12 +526,12 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
         tmem_st_wait();
         fence_proxy_async();
         tc_fence_before();
-        mbar_arrive(&bar[P2_SBFULL]);
+        warp_arrive(&bar[P2_SBFULL]);
         for (int n = 0; n < ncj; ++n) {
             const int s = n & 1;
             // D = U + Y for this warp's 64 columns (the same U for both runs)
-            if (!mbar_wait(&bar[P2_DFULL], n & 1, abort_flag)) break;
-            if (!mbar_wait(&bar[P2_FULL + s], (n >> 1) & 1, abort_flag)) break;
+            if (!warp_wait(&bar[P2_DFULL], n & 1, abort_flag)) break;
+            if (!warp_wait(&bar[P2_FULL + s], (n >> 1) & 1, abort_flag)) break;
             if (threadIdx.x == 0) EFLA_TR2(41, n);
             tc_fence_after();
             const unsigned char *urow = sm + s * P2_STAGE + 6 * SLOT + drow * 256;
@@ -544,10 +554,10 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             }
             fence_proxy_async();
             tc_fence_before();
-            mbar_arrive(&bar[P2_DELTA]);
+            warp_arrive(&bar[P2_DELTA]);
             if (threadIdx.x == 0) EFLA_TR2(42, n);
             // S out of TMEM: the bf16 operand of the next chunk, or the final states
-            if (!mbar_wait(&bar[P2_SFULL], n & 1, abort_flag)) break;
+            if (!warp_wait(&bar[P2_SFULL], n & 1, abort_flag)) break;
             if (threadIdx.x == 0) EFLA_TR2(43, n);
             tc_fence_after();
             float *dst = n == ncj - 1 ? (run == 0 ? job.sl : job.sl2) : nullptr;
@@ -572,7 +582,7 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             if (n < ncj - 1) {
                 fence_proxy_async();
                 tc_fence_before();
-                mbar_arrive(&bar[P2_SBFULL]);
+                warp_arrive(&bar[P2_SBFULL]);
                 if (threadIdx.x == 0) EFLA_TR2(44, n);
             }
         }
@@ -688,12 +698,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar[B_FULLB + s], 1);
             mbar_init(&bar[B_EMPTYA + s], 1);
             mbar_init(&bar[B_EMPTYB + s], 1);
-            mbar_init(&bar[B_OREAD + s], 128);
+            mbar_init(&bar[B_OREAD + s], 4);  // the 4 O warps
             mbar_init(&bar[B_OFULL + s], 1);
         }
-        mbar_init(&bar[B_SBFULL], 256);
+        mbar_init(&bar[B_SBFULL], 8);  // one arrival per converter warp
         mbar_init(&bar[B_DFULL], 1);
-        mbar_init(&bar[B_DELTA], 128);
+        mbar_init(&bar[B_DELTA], 4);  // the 4 D warps
         mbar_init(&bar[B_SFULL], 1);
         mbar_init(&bar[B_DRAIN], 1);
         fence_mbar_init();
@@ -746,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             write_split32(sm + OFF_SB, 2 * SLOT, row, 4 * cpart, x);
             fence_proxy_async();
             tc_fence_before();
-            mbar_arrive(&bar[B_SBFULL]);
+            warp_arrive(&bar[B_SBFULL]);
         }
         // A state-row warp (quads 2, 3) leaves the loop on its own when a wait
         // fails: no barrier inside the loop ties it to the others.  The O
@@ -761,8 +771,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c = row - 64;
                 // (the stage's own barrier too: U landed by the bulk copy is
                 // visible to the threads that observe that barrier's phase)
-                if (!mbar_wait(&bar[B_FULLB + b], (n >> 1) & 1, abort_flag)) break;
-                if (!mbar_wait(&bar[B_DFULL], n & 1, abort_flag)) break;
+                if (!warp_wait(&bar[B_FULLB + b], (n >> 1) & 1, abort_flag)) break;
+                if (!warp_wait(&bar[B_DFULL], n & 1, abort_flag)) break;
                 if (row == 64 && cpart == 0) EFLA_TR(28, n);
                 tc_fence_after();
                 uint32_t r[32], r2[32];
@@ -786,10 +796,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 write_split32(sm + OFF_DB + b * 2 * SLOT, SLOT, c, 4 * cpart, x);
                 fence_proxy_async();
                 tc_fence_before();
-                mbar_arrive(&bar[B_DELTA]);
+                warp_arrive(&bar[B_DELTA]);
                 if (row == 64 && cpart == 0) EFLA_TR(11, n);
             }
-            const bool ok = mbar_wait(&bar[B_SFULL], n & 1, abort_flag);
+            const bool ok = warp_wait(&bar[B_SFULL], n & 1, abort_flag);
             if (row == 64 && cpart == 0) EFLA_TR(12, n);
             if (!ok && dwarp) break;
             if (ok) {
@@ -806,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (row == 64 && cpart == 0) EFLA_TR(31, n);
                 fence_proxy_async();
                 tc_fence_before();
-                mbar_arrive(&bar[B_SBFULL]);
+                warp_arrive(&bar[B_SBFULL]);
                 if (row == 64 && cpart == 0) EFLA_TR(13, n);
             }
             if (ok && n == ncj - 1 && job.sl) {
@@ -831,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_wait(r);
                     tmem_ld_wait(r2);
                     tc_fence_before();
-                    mbar_arrive(&bar[B_OREAD + b]);
+                    warp_arrive(&bar[B_OREAD + b]);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) + __uint_as_float(r2[i]));
                     if (row == 0 && cpart == 0) EFLA_TR(14, n);
