@@ -439,7 +439,7 @@ struct SegPlan {
 // chunk (no Q, M or O):
 //   Y  = [-W; -W] [S_hi | S_lo]            (tcgen05, M=128 N=256 K=128)
 //   D  = U + Y_hi + Y_lo                   (both halves of the 128 columns)
-//   S += K^T [D_hi | D_lo]                 (tcgen05, M=128 N=256 K=64)
+//   S += K^T (D_hi + D_lo)                 (tcgen05, M=128 N=128 K=64, hi then lo)
 // -W is stacked twice so that every row of Y sits in two TMEM lanes (i and
 // 64 + i): an M = 128 product costs what an M = 64 one does, and all 32
 // lanes of every read-out warp then carry a row (lanes 0-63 the run from
@@ -448,18 +448,20 @@ struct SegPlan {
 //   two stages of W0 W0 W1 W1 K0 K1 U (U: this d_v half, 64 rows x 256 B)
 //   S bf16: hi box 0, hi box 1, lo box 0, lo box 1 (128 rows x 64 columns each)
 //   D bf16: hi box 0, hi box 1, lo box 0, lo box 1 (64 rows x 64 columns each)
-// The hi and lo halves of S and D sit side by side as one N = 256 operand
-// (as in the single run): the state is S_a + S_b, and Y is read out as
-// Y_hi + Y_lo.
-// TMEM: S [0, 256) = [S_a | S_b], Y [256, 512) = [Y_hi | Y_lo], each half
-// 128 columns [run from zero | run from the identity].
+// The hi and lo halves of S sit side by side as one N = 256 operand of Y
+// (as in the single run), and Y is read out as Y_hi + Y_lo.  The state
+// update keeps one accumulator (D_hi, then D_lo): the S read-out of 128
+// columns per row is the longest step here, and a second accumulator would
+// add a load and an add per element to it.
+// TMEM: S [0, 128) [run from zero | run from the identity], Y [256, 512) =
+// [Y_hi | Y_lo], each half 128 columns [zero | identity].
 constexpr uint32_t P2_STAGE = 8 * SLOT;
 constexpr uint32_t P2_SB = 2 * P2_STAGE, P2_DB = P2_SB + 8 * SLOT, P2_BAR = P2_DB + 4 * SLOT;
 static_assert(P2_BAR <= OFF_BAR, "paired runs keep their barriers inside the serial kernel's layout");
 static_assert(P2_BAR + 128 + 1024 <= SMEM_BYTES, "paired runs fit the serial kernel's shared memory");
 constexpr uint32_t T2_S = 0, T2_Y = 256, T2_COLS = 512;
 constexpr uint32_t ID2_Y = ptx::idesc_bf16(128, 256, false, true);
-constexpr uint32_t ID2_S = ptx::idesc_bf16(128, 256, true, true);
+constexpr uint32_t ID2_S = ptx::idesc_bf16(128, 128, true, true);
 enum : int { P2_FULL = 0, P2_EMPTY = 2, P2_SBFULL = 4, P2_DFULL = 5, P2_DELTA = 6, P2_SFULL = 7, P2_DRAIN = 8 };
 
 __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &tm_k, const unsigned char *ws,
@@ -518,9 +520,6 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
             tmem_st32(tl + T2_S + 64 * run + 32 * hh, r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = 0u;
-            tmem_st32(tl + T2_S + 128 + 64 * run + 32 * hh, r);
             write_split32(sm + P2_SB + run * 2 * SLOT, 4 * SLOT, row, 4 * hh, x);
         }
         tmem_st_wait();
@@ -563,13 +562,10 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             float *dst = n == ncj - 1 ? (run == 0 ? job.sl : job.sl2) : nullptr;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                uint32_t r[32], r2[32];
-                tmem_ld32(tl + T2_S + 64 * run + 32 * hh, r);         // S_a
-                tmem_ld32(tl + T2_S + 128 + 64 * run + 32 * hh, r2);  // S_b
+                uint32_t r[32];
+                tmem_ld32(tl + T2_S + 64 * run + 32 * hh, r);
                 tmem_ld_wait(r);
-                tmem_ld_wait(r2);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]) + __uint_as_float(r2[i]);
+                as_float32(r, x);
                 if (n < ncj - 1) {
                     write_split32(sm + P2_SB + run * 2 * SLOT, 4 * SLOT, row, 4 * hh, x);
                 } else if (dst) {
@@ -609,12 +605,15 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             if (!warp_wait(&bar[P2_DELTA], n & 1, abort_flag)) break;
             tc_fence_after();
             if (leader) EFLA_TR2(45, n);
-            if (leader) {  // S += K^T [D_hi | D_lo]: 4 k-steps over the chunk
+            if (leader) {  // S += K^T (D_hi + D_lo): 4 k-steps over the chunk, hi then lo
                 const uint64_t dKt = sdesc_sw128(st + 4 * SLOT, SLOT, 1024);
                 const uint64_t dD = sdesc_sw128(sbase + P2_DB, SLOT, 1024);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + T2_S, dKt + ((kk * 2048) >> 4), dD + ((kk * 2048) >> 4), ID2_S, 1);
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + T2_S, dKt + ((kk * 2048) >> 4), dD + ((part * 2 * SLOT + kk * 2048) >> 4),
+                                 ID2_S, 1);
                 mma_commit(&bar[P2_SFULL]);
                 mma_commit(&bar[P2_EMPTY + s]);
             }
