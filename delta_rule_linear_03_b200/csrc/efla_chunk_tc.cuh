@@ -419,7 +419,8 @@ struct SegJob {
     const float *s0;  // [B*H][d_k][d_v] fp32 (s0_kind 1)
     float *sl;        // final state, [B*H][d_k][d_v] fp32, or null
     int pair;         // run from zero and from the identity together (no outputs):
-                      // final states to sl (from zero) and sl2 (from the identity)
+                      // final state from zero to sl, and the segment's map
+                      // (final state from the identity minus sl) to sl2
     float *sl2;
 };
 constexpr int kMaxJobs = 16;
@@ -526,6 +527,7 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
         fence_proxy_async();
         tc_fence_before();
         warp_arrive(&bar[P2_SBFULL]);
+        bool fin = false;  // this warp reached the final states
         for (int n = 0; n < ncj; ++n) {
             const int s = n & 1;
             // D = U + Y for this warp's 64 columns (the same U for both runs)
@@ -559,27 +561,58 @@ __device__ __forceinline__ void pair_run(unsigned char *sm, const CUtensorMap &t
             if (!warp_wait(&bar[P2_SFULL], n & 1, abort_flag)) break;
             if (threadIdx.x == 0) EFLA_TR2(43, n);
             tc_fence_after();
-            float *dst = n == ncj - 1 ? (run == 0 ? job.sl : job.sl2) : nullptr;
+            if (n == ncj - 1) {  // the final states are read after the loop
+                fin = true;
+                break;
+            }
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t r[32];
                 tmem_ld32(tl + T2_S + 64 * run + 32 * hh, r);
                 tmem_ld_wait(r);
                 as_float32(r, x);
-                if (n < ncj - 1) {
-                    write_split32(sm + P2_SB + run * 2 * SLOT, 4 * SLOT, row, 4 * hh, x);
-                } else if (dst) {
-                    float *d = dst + ((size_t)bh * DK + row) * DK + j0 + 32 * hh;
-#pragma unroll
-                    for (int c = 0; c < 32; c += 4)
-                        *reinterpret_cast<float4 *>(d + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
-                }
+                write_split32(sm + P2_SB + run * 2 * SLOT, 4 * SLOT, row, 4 * hh, x);
             }
-            if (n < ncj - 1) {
-                fence_proxy_async();
-                tc_fence_before();
-                warp_arrive(&bar[P2_SBFULL]);
-                if (threadIdx.x == 0) EFLA_TR2(44, n);
+            fence_proxy_async();
+            tc_fence_before();
+            warp_arrive(&bar[P2_SBFULL]);
+            if (threadIdx.x == 0) EFLA_TR2(44, n);
+        }
+        // Final states: S(0) to sl, and the segment's map M = S(I) - S(0) to
+        // sl2 (the segment chain's operand).  Every converter warp reaches this
+        // vote, also after a failed wait, so the named barrier below cannot
+        // miss a warp; after a failure nobody writes.  The run-from-zero warps
+        // park their rows in shared memory (the S operand tiles: every product
+        // has completed by now) for the identity-run warps of the same lanes.
+        if (!bar_any(4, 256, !fin || *abort_flag)) {
+            float *park = reinterpret_cast<float *>(sm + P2_SB);  // 128 rows x 32 columns
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t r[32];
+                tmem_ld32(tl + T2_S + 64 * run + 32 * hh, r);
+                tmem_ld_wait(r);
+                as_float32(r, x);
+                float *pk = park + row * 32;
+                if (run == 0) {
+                    float *d = job.sl + ((size_t)bh * DK + row) * DK + j0 + 32 * hh;
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 v = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+                        *reinterpret_cast<float4 *>(d + c) = v;
+                        *reinterpret_cast<float4 *>(pk + c) = v;
+                    }
+                }
+                named_bar(4, 256);  // the run-from-zero half-rows are parked
+                if (run == 1) {
+                    float *d = job.sl2 + ((size_t)bh * DK + row) * DK + j0 + 32 * hh;
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 z = *reinterpret_cast<const float4 *>(pk + c);
+                        *reinterpret_cast<float4 *>(d + c) =
+                            make_float4(x[c] - z.x, x[c + 1] - z.y, x[c + 2] - z.z, x[c + 3] - z.w);
+                    }
+                }
+                named_bar(4, 256);  // read before the next half overwrites the park
             }
         }
     } else if (warp == 8) {
@@ -1417,9 +1450,9 @@ inline int sm_count() {
 // otherwise 1 (a single pass).
 constexpr int kMinSegChunks = 16;
 // The time of a paired-run chunk (pair_run) relative to a single run's, in
-// per cent (clock64 traces: 4.45k cycles per paired-run chunk on the
-// long-context prefill against 3.28k per single-run chunk on lm340m).
-constexpr long kPairCost = 136;
+// per cent (clock64 traces: 4.29k cycles per paired-run chunk on the
+// long-context prefill against 3.12k per single-run chunk on lm340m).
+constexpr long kPairCost = 137;
 inline int segments(long bh, int nc) {
     const long sms = sm_count();
     int best = 1;
@@ -1488,21 +1521,24 @@ __global__ void __launch_bounds__(256) affine_step_kernel(const float *__restric
 }
 
 // The whole segment chain in one launch: for r = 1 .. steps,
-//   X(r+1) = (SI(r) - SZ(r)) X(r) + SZ(r),
-// with X(1) given and consecutive SI, SZ and X states `stride` floats apart.
-// Column block j of X(r+1) needs only column block j of X(r), so CTA
-// (bh, column block of 32) walks every step on its own, its X block resident
-// in shared memory.  Thread (ty, tx) owns four rows x four columns; the
-// reduction runs in slabs of 32, the next slab of SI - SZ loaded into
-// registers while the current one is used.
+//   X(r+1) = M(r) X(r) + SZ(r),
+// with X(1) given, M(r) the segment maps written by the paired runs, and
+// consecutive M, SZ and X states `stride` floats apart.  Column block j of
+// X(r+1) needs only column block j of X(r), so CTA (bh, column block of 32)
+// walks every step on its own, its X block resident in shared memory.  A
+// step's whole M(r) (d x d) is loaded at once into shared memory, the next
+// step's into registers while the current one is used, so each step waits
+// for at most one memory round trip.  Thread (ty, tx) owns four rows x four
+// columns.
 template <int D>
-__global__ void __launch_bounds__(256) affine_chain_kernel(const float *__restrict__ SI, const float *__restrict__ SZ,
+__global__ void __launch_bounds__(256) affine_chain_kernel(const float *__restrict__ M, const float *__restrict__ SZ,
                                                            float *__restrict__ X, int steps, size_t stride) {
     static_assert(D % 32 == 0 && D <= 128, "D in {32, 64, 128}");
-    constexpr int NS = D / 32;              // slabs per step
-    constexpr int NE = D * 32 / 256;        // slab elements per thread
-    __shared__ float Ms[D][33];
-    __shared__ __align__(16) float Xs[D][36];
+    constexpr int LM = D + 1;                 // row stride of M in shared memory (odd: column reads spread over banks)
+    constexpr int NF = D * D / 4 / 256;       // float4s of one step's M per thread
+    extern __shared__ __align__(16) float chain_sm[];
+    float *Ms = chain_sm;                                          // D x LM
+    float(*Xs)[36] = reinterpret_cast<float(*)[36]>(chain_sm + ((D * LM + 3) & ~3));  // D x 32 (+4)
     const size_t base = (size_t)blockIdx.x * D * D;
     const int cb = 32 * blockIdx.y, tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
     const bool active = 4 * ty < D;
@@ -1511,60 +1547,70 @@ __global__ void __launch_bounds__(256) affine_chain_kernel(const float *__restri
         const int r = e >> 5, c = e & 31;
         Xs[r][c] = X[base + (size_t)r * D + cb + c];
     }
-    float mreg[NE];
-    auto fetch = [&](int step, int k0) {  // slab k0 of SI(step) - SZ(step)
-        const float *si = SI + (size_t)step * stride + base, *sz = SZ + (size_t)step * stride + base;
+    float4 mreg[NF];
+    auto fetch = [&](int step) {
+        const float4 *m = reinterpret_cast<const float4 *>(M + (size_t)step * stride + base);
 #pragma unroll
-        for (int x = 0; x < NE; ++x) {
-            const int e = tid + 256 * x, r = e >> 5, c = e & 31;
-            const size_t a = (size_t)r * D + k0 + c;
-            mreg[x] = si[a] - sz[a];
-        }
+        for (int x = 0; x < NF; ++x) mreg[x] = m[tid + 256 * x];
     };
-    if (steps > 0) fetch(0, 0);
+    if (steps > 0) fetch(0);
     for (int step = 0; step < steps; ++step) {
-        float acc[4][4] = {};
-        for (int s = 0; s < NS; ++s) {
-            __syncthreads();  // the previous slab (and, at s = 0, the X block) fully used / written
+        __syncthreads();  // the previous step is done with Ms (and, at step 0, Xs is written)
 #pragma unroll
-            for (int x = 0; x < NE; ++x) {
-                const int e = tid + 256 * x;
-                Ms[e >> 5][e & 31] = mreg[x];
+        for (int x = 0; x < NF; ++x) {
+            const int e = 4 * (tid + 256 * x), r = e / D, c = e % D;
+            float *d = Ms + r * LM + c;
+            d[0] = mreg[x].x;
+            d[1] = mreg[x].y;
+            d[2] = mreg[x].z;
+            d[3] = mreg[x].w;
+        }
+        if (step + 1 < steps) fetch(step + 1);
+        // this step's SZ block of the thread, loaded during the product
+        float szr[4][4];
+        if (active) {
+            const float *sz = SZ + (size_t)step * stride + base;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 v = *reinterpret_cast<const float4 *>(sz + (size_t)(4 * ty + i) * D + cb + 4 * tx);
+                szr[i][0] = v.x, szr[i][1] = v.y, szr[i][2] = v.z, szr[i][3] = v.w;
             }
-            if (s + 1 < NS) fetch(step, 32 * (s + 1));
-            else if (step + 1 < steps) fetch(step + 1, 0);
-            __syncthreads();
-            if (active) {
+        }
+        __syncthreads();
+        float acc[4][4] = {};
+        if (active) {
 #pragma unroll 8
-                for (int k = 0; k < 32; ++k) {
-                    const float4 b = *reinterpret_cast<const float4 *>(&Xs[32 * s + k][4 * tx]);
+            for (int k = 0; k < D; ++k) {
+                const float4 b = *reinterpret_cast<const float4 *>(&Xs[k][4 * tx]);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float a = Ms[4 * ty + i][k];
-                        acc[i][0] = fmaf(a, b.x, acc[i][0]);
-                        acc[i][1] = fmaf(a, b.y, acc[i][1]);
-                        acc[i][2] = fmaf(a, b.z, acc[i][2]);
-                        acc[i][3] = fmaf(a, b.w, acc[i][3]);
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const float a = Ms[(4 * ty + i) * LM + k];
+                    acc[i][0] = fmaf(a, b.x, acc[i][0]);
+                    acc[i][1] = fmaf(a, b.y, acc[i][1]);
+                    acc[i][2] = fmaf(a, b.z, acc[i][2]);
+                    acc[i][3] = fmaf(a, b.w, acc[i][3]);
                 }
             }
         }
         __syncthreads();  // every thread is done reading Xs of this step
         if (active) {
-            const float *sz = SZ + (size_t)step * stride + base;
             float *out = X + (size_t)(step + 1) * stride + base;
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = 4 * ty + i, c = 4 * tx + j;
-                    const float y = acc[i][j] + sz[(size_t)r * D + cb + c];
-                    out[(size_t)r * D + cb + c] = y;
-                    Xs[r][c] = y;
-                }
+            for (int i = 0; i < 4; ++i) {
+                const int r = 4 * ty + i;
+                const float4 y = make_float4(acc[i][0] + szr[i][0], acc[i][1] + szr[i][1], acc[i][2] + szr[i][2],
+                                             acc[i][3] + szr[i][3]);
+                *reinterpret_cast<float4 *>(out + (size_t)r * D + cb + 4 * tx) = y;
+                *reinterpret_cast<float4 *>(&Xs[r][4 * tx]) = y;
+            }
         }
     }
     EFLA_GT_END(4);
+}
+// Shared memory of affine_chain_kernel<D>.
+template <int D>
+constexpr size_t chain_smem_bytes() {
+    return (size_t)(((D * (D + 1) + 3) & ~3) + D * 36) * sizeof(float);
 }
 
 template <typename Tout>
@@ -1578,7 +1624,8 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
         return EFLA_ERR_CUDA;
     CUtensorMap mv;
     if (!make_map_bf16_sw128(&mv, v, bh, L)) return EFLA_ERR_CUDA;
-    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES) || !ensure_smem<chunk_prep_tc_kernel>(P_SMEM))
+    if (!ensure_smem<chunk_tc_kernel<Tout>>(SMEM_BYTES) || !ensure_smem<chunk_prep_tc_kernel>(P_SMEM) ||
+        !ensure_smem<affine_chain_kernel<DK>>(chain_smem_bytes<DK>()))
         return EFLA_ERR_CUDA;
     const long grid = bh * NSPLIT;
     const int nc = (L + C - 1) / C;
@@ -1633,8 +1680,13 @@ inline efla_status_t launch(const void *q, const void *k, const void *v, const f
     for (int r = 1; r <= P - 2; ++r)
         plan.job[plan.njobs++] = SegJob{first(r), first(r + 1) - first(r), 0, 0, nullptr, SZ(r), 1, SI(r)};
     if (!run(plan)) return EFLA_ERR_CUDA;
-    // the segment chain, one launch: Sin(r + 1) = (SI(r) - SZ(r)) Sin(r) + SZ(r)
-    affine_chain_kernel<DK><<<dim3((unsigned)bh, DK / 32), 256, 0, st>>>(SI(1), SZ(1), Sin(1), P - 2, sb);
+    // the segment chain, one launch: Sin(r + 1) = M(r) Sin(r) + SZ(r), with
+    // the paired runs' maps M(r) = S(I)(r) - S(0)(r) in the SI buffers
+    // (an ordinary launch: as a programmatic dependent of pass A its first
+    // CTAs were scheduled two to an SM on the SMs pass A leaves free, and the
+    // chain took 40 instead of 23 µs)
+    affine_chain_kernel<DK><<<dim3((unsigned)bh, DK / 32), 256, chain_smem_bytes<DK>(), st>>>(SI(1), SZ(1), Sin(1),
+                                                                                           P - 2, sb);
     if (cudaGetLastError() != cudaSuccess) return EFLA_ERR_CUDA;
     // pass B
     plan.njobs = 0;
