@@ -84,11 +84,11 @@ def cpu_model() -> str:
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
 # long-context efla_chunk_fwd call, all launches: an ncu capture of the same
 # call at L = 16384 (16 heads, the same segmented kernels and plan shape)
-# measured 734.3 MB read + 274.6 MB written per call; the per-chunk work and
-# images scale with L, so the full call moves about 4 x 1008.9 MB.  It is
+# measured 733.3 MB read + 274.0 MB written per call; the per-chunk work and
+# images scale with L, so the full call moves about 4 x 1007.3 MB.  It is
 # 3.7 x the algorithmic bytes: the per-chunk workspace image (-W, M, U)
 # makes a round trip, and pass A and pass B both read the middle segments.
-LONGCTX_TRAFFIC = 4 * 1008.9e6
+LONGCTX_TRAFFIC = 4 * 1007.3e6
 
 
 def chunk_bytes(B, H, L, d, esize, esize_o, s0: bool, sl: bool = True):
