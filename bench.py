@@ -712,11 +712,9 @@ def bench_e2e(efla, dev, x, args, world):
     """The same metric through the public API from pinned host buffers:
     every step copies q, k, v, beta host->device, runs efla_chunk_fwd and
     copies o and S_L device->host.  Steps are pipelined the way a serving
-    loop would run them: copy-in, compute and copy-out streams and two device
-    buffer sets, so that step i+1's inputs cross PCIe while step i computes
-    and step i-1's outputs come back (PCIe is full duplex).  The inputs go
-    over two copy-in streams (q and beta, k and v), so two copy engines share
-    the host-to-device direction.  Each
+    loop would run them: three streams (copy in, compute, copy out) and two
+    device buffer sets, so that step i+1's inputs cross PCIe while step i
+    computes and step i-1's outputs come back (PCIe is full duplex).  Each
     step still moves all of its own inputs and outputs inside the timed
     region; a buffer set is refilled only after the step that used it has
     been copied out."""
@@ -728,24 +726,18 @@ def bench_e2e(efla, dev, x, args, world):
     do = [torch.empty(B, H, L, d, dtype=torch.float32, device=dev) for _ in range(2)]
     dS = [torch.empty(B, H, d, d, dtype=torch.float32, device=dev) for _ in range(2)]
     ws = torch.empty(max(efla.workspace_size(hq.dtype, B, H, L, d, d), 16), dtype=torch.uint8, device=dev)
-    s_in = [torch.cuda.Stream(dev) for _ in range(2)]
-    s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [[torch.cuda.Event() for _ in range(2)] for _ in range(2)]  # [copy stream][buffer set]
-    ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(2))
-    srcs = (hq, hk, hv, hb)
-    split = ((0, 3), (1, 2))  # copy stream 0: q, beta; copy stream 1: k, v
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
     def step(i):
         b = i % 2
-        for c, idx in enumerate(split):
-            with torch.cuda.stream(s_in[c]):
-                s_in[c].wait_event(ev_comp[b])   # step i-2 has finished reading this input set
-                for j in idx:
-                    din[b][j].copy_(srcs[j], non_blocking=True)
-                ev_in[c][b].record(s_in[c])
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_comp[b])       # step i-2 has finished reading this input set
+            for dst, src in zip(din[b], (hq, hk, hv, hb)):
+                dst.copy_(src, non_blocking=True)
+            ev_in[b].record(s_in)
         with torch.cuda.stream(s_comp):
-            for c in range(2):
-                s_comp.wait_event(ev_in[c][b])
+            s_comp.wait_event(ev_in[b])
             s_comp.wait_event(ev_out[b])      # step i-2's outputs have left this output set
             efla.chunk_fwd(*din[b], None, o=do[b], S_L=dS[b], workspace=ws)
             ev_comp[b].record(s_comp)
@@ -757,11 +749,11 @@ def bench_e2e(efla, dev, x, args, world):
 
     def run(n):
         cur = torch.cuda.current_stream(dev)
-        for s in (*s_in, s_comp, s_out):
+        for s in (s_in, s_comp, s_out):
             s.wait_stream(cur)
         for i in range(n):
             step(i)
-        for s in (*s_in, s_comp, s_out):
+        for s in (s_in, s_comp, s_out):
             cur.wait_stream(s)
 
     run(3)
@@ -786,7 +778,7 @@ def bench_e2e(efla, dev, x, args, world):
     d2h = ho[0].numel() * ho[0].element_size() + hS[0].numel() * hS[0].element_size()
     return {"value": world * B * L * n / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n, "single_step_ms": one_ms,
-            "pipeline": "2 copy-in streams, compute and copy-out streams, 2 buffer sets; steps overlap"}
+            "pipeline": "3 streams (copy in / compute / copy out), 2 buffer sets; steps overlap"}
 
 
 def run_profile_case(case: str, calls: int, seq_len=None):
